@@ -1,0 +1,184 @@
+"""Seeded synthetic inputs for the MALA workloads.
+
+This module holds no attention arithmetic: it only draws tensors.  Both the CUDA path
+(tests, bench) and the CPU oracle consume exactly these values.  Every draw comes from
+numpy's Philox counter-based generator keyed by (config seed, tensor id, chunk), so a
+tensor is reproducible on any machine with the same numpy.
+
+All tensors are returned as float32 numpy arrays whose values are already rounded to
+the compute dtype (round-to-nearest-even to bf16 for bf16 workloads), so converting
+them to bf16 on the device is exact and the oracle widens the same values to fp64.
+
+Workloads (the attention page's own experiments run on real model states, which are not
+available; these synthetic distributions stand in for them):
+
+* ``tiny256``     B=1, H=2, H_kv=2, L=256, d=64, fp32; Q, K, V ~ N(0, 1)
+* ``peaked1k``    B=2, H=8, H_kv=2, L=1024, d=128, bf16; K ~ N(0, 1); query row t is
+                  3.0 x the mean of 4 keys drawn uniformly (with replacement) from its
+                  causal prefix [0, t] of its own KV head, plus N(0, 1) noise
+* ``mixed8k``     B=1, H=16, H_kv=4, L=8192, d=128, bf16; heads 0-7 peaked as above,
+                  heads 8-15 diffuse (Q ~ N(0, 1))
+* ``sinkband32k`` B=1, H=32, H_kv=8, L=32768, d=128, bf16; K ~ N(0, 1) with key 0
+                  scaled by 4 (attention sink); q_t = 0.5 u_t + sqrt(0.75) n_t with
+                  u_t = (1/sqrt(w)) sum_{s=t-w}^{t-1} K_s, w = min(64, t), u_0 = 0
+* ``decode128k``  B=4, H=32, H_kv=8, N_k=131072, d=128, bf16; K, V, q ~ N(0, 1); per
+                  (b, KV head) 16 distinct random positions get a planted key
+                  3.0 * sqrt(d) * q_h / |q_h| + N(0, 1), h cycling over the group's heads
+
+V ~ N(0, 1) everywhere; dO is a Rademacher (+-1) probe.
+"""
+
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, field
+
+import numpy as np
+
+# tensor ids used in the Philox key
+_Q, _K, _V, _DO, _POS, _NOISE, _PLANT = 1, 2, 3, 4, 5, 6, 7
+
+
+@dataclass(frozen=True)
+class Workload:
+    name: str
+    B: int
+    H: int
+    H_kv: int
+    L: int
+    d: int
+    dtype: str  # "bf16" or "fp32"
+    structure: str  # normal | peaked | half_peaked | sink_band | planted
+    seed: int
+    decode: bool = False
+    taus: tuple = field(default=(1.0,))
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.d)
+
+
+WORKLOADS = {
+    "tiny256": Workload("tiny256", 1, 2, 2, 256, 64, "fp32", "normal", 0, taus=(0.0, 1.0)),
+    "peaked1k": Workload("peaked1k", 2, 8, 2, 1024, 128, "bf16", "peaked", 1),
+    "mixed8k": Workload("mixed8k", 1, 16, 4, 8192, 128, "bf16", "half_peaked", 2,
+                        taus=(1.0, 0.0, 1e-4, 1e-3)),
+    "sinkband32k": Workload("sinkband32k", 1, 32, 8, 32768, 128, "bf16", "sink_band", 3),
+    "decode128k": Workload("decode128k", 4, 32, 8, 131072, 128, "bf16", "planted", 4,
+                           decode=True),
+}
+
+
+def _rng(seed: int, tensor: int, chunk: int = 0) -> np.random.Generator:
+    return np.random.Generator(np.random.Philox(key=[seed, tensor * 1_000_003 + chunk]))
+
+
+def round_bf16(x: np.ndarray) -> np.ndarray:
+    """Round float32 values to the nearest bf16 (ties to even); returns float32."""
+    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32)
+    r = (u + np.uint32(0x7FFF) + ((u >> np.uint32(16)) & np.uint32(1))) & np.uint32(0xFFFF0000)
+    return r.view(np.float32)
+
+
+def _round(x: np.ndarray, dtype: str) -> np.ndarray:
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    return round_bf16(x) if dtype == "bf16" else x
+
+
+def normal(seed: int, tensor: int, shape, dtype: str, chunk_axis0: bool = True) -> np.ndarray:
+    """N(0, 1) draws of ``shape``, generated in chunks along axis 0 (one key per chunk)."""
+    out = np.empty(shape, dtype=np.float32)
+    if chunk_axis0 and len(shape) > 1:
+        for c in range(shape[0]):
+            out[c] = _rng(seed, tensor, c).standard_normal(shape[1:], dtype=np.float32)
+    else:
+        out[...] = _rng(seed, tensor).standard_normal(shape, dtype=np.float32)
+    return _round(out, dtype)
+
+
+def rademacher(seed: int, tensor: int, shape) -> np.ndarray:
+    bits = _rng(seed, tensor).integers(0, 2, size=shape, dtype=np.int8)
+    return (bits.astype(np.float32) * 2.0 - 1.0)
+
+
+def _peaked_queries(K: np.ndarray, heads, H: int, seed: int, dtype: str,
+                    noise: np.ndarray) -> np.ndarray:
+    """q_t = 3.0 * mean of 4 keys drawn from [0, t] of the head's KV head + noise."""
+    B, L, Hkv, d = K.shape
+    G = H // Hkv
+    rng = _rng(seed, _POS)
+    out = {}
+    t = np.arange(L)
+    for h in heads:
+        g = h // G
+        u = rng.random((B, L, 4))
+        pos = np.minimum((u * (t[None, :, None] + 1)).astype(np.int64), t[None, :, None])
+        keys = K[np.arange(B)[:, None, None], pos, g]  # [B, L, 4, d]
+        out[h] = 3.0 * keys.astype(np.float64).mean(axis=2) + noise[:, :, h].astype(np.float64)
+    return out
+
+
+def make_training(w: Workload, L: int | None = None) -> dict:
+    """Q, K, V, dO for a training-shape workload (optionally with a different L)."""
+    assert not w.decode
+    L = w.L if L is None else L
+    B, H, Hkv, d = w.B, w.H, w.H_kv, w.d
+    K = normal(w.seed, _K, (B, L, Hkv, d), w.dtype)
+    V = normal(w.seed, _V, (B, L, Hkv, d), w.dtype)
+    dO = rademacher(w.seed, _DO, (B, L, H, d))
+    if w.structure == "normal":
+        Q = normal(w.seed, _Q, (B, L, H, d), w.dtype)
+    elif w.structure in ("peaked", "half_peaked"):
+        noise = normal(w.seed, _NOISE, (B, L, H, d), "fp32")
+        heads = range(H) if w.structure == "peaked" else range(H // 2)
+        Q = noise.copy()  # diffuse heads: Q ~ N(0, 1)
+        for h, q in _peaked_queries(K, heads, H, w.seed, w.dtype, noise).items():
+            Q[:, :, h] = q
+        Q = _round(Q, w.dtype)
+    elif w.structure == "sink_band":
+        K = K.copy()
+        K[:, 0] = _round(K[:, 0] * 4.0, w.dtype)
+        n = normal(w.seed, _NOISE, (B, L, H, d), "fp32")
+        cs = np.zeros((B, L + 1, Hkv, d), dtype=np.float64)
+        np.cumsum(K, axis=1, dtype=np.float64, out=cs[:, 1:])
+        t = np.arange(L)
+        wlen = np.minimum(64, t)
+        win = cs[:, t] - cs[:, t - wlen]  # sum of K_{t-w} .. K_{t-1}
+        u = win / np.sqrt(np.maximum(wlen, 1))[None, :, None, None]
+        G = H // Hkv
+        Q = np.empty((B, L, H, d), dtype=np.float32)
+        for h in range(H):
+            Q[:, :, h] = 0.5 * u[:, :, h // G] + math.sqrt(0.75) * n[:, :, h]
+        Q = _round(Q, w.dtype)
+    else:
+        raise ValueError(w.structure)
+    return {"Q": Q, "K": K, "V": V, "dO": dO}
+
+
+def make_decode(w: Workload, Nk: int | None = None, B: int | None = None) -> dict:
+    """q [B,H,d] and the KV cache K, V [B,Nk,Hkv,d] for a decode workload."""
+    assert w.decode
+    Nk = w.L if Nk is None else Nk
+    B = w.B if B is None else B
+    H, Hkv, d = w.H, w.H_kv, w.d
+    G = H // Hkv
+    q = normal(w.seed, _Q, (B, H, d), w.dtype)
+    K = normal(w.seed, _K, (B, Nk, Hkv, d), w.dtype)
+    V = normal(w.seed, _V, (B, Nk, Hkv, d), w.dtype)
+    rng = _rng(w.seed, _PLANT)
+    n_plant = min(16, Nk)
+    for b in range(B):
+        for g in range(Hkv):
+            pos = rng.choice(Nk, size=n_plant, replace=False)
+            for r, p in enumerate(pos):
+                h = g * G + (r % G)
+                qh = q[b, h].astype(np.float64)
+                key = 3.0 * math.sqrt(d) * qh / np.linalg.norm(qh) + rng.standard_normal(d)
+                K[b, p, g] = _round(key.astype(np.float32), w.dtype)
+    return {"q": q, "K": K, "V": V}
+
+
+def small_training(B=1, H=2, Hkv=1, L=192, d=64, dtype="bf16", structure="normal", seed=11):
+    """A small ad-hoc training workload (parity tests: ragged tails, GQA, d=64)."""
+    w = Workload(f"adhoc{L}", B, H, Hkv, L, d, dtype, structure, seed)
+    return w, make_training(w)
