@@ -1,0 +1,136 @@
+/*
+ * mala.h - C ABI of the B200 (sm_100a) MassAlloc Attention (MALA) library.
+ *
+ * MALA is causal softmax attention that computes every legal causal QK^T score tile
+ * and then runs the post-score work of a tile (exp, P.V and, in backward, the
+ * dP/dS/dQ/dK/dV products) only when the tile's normalised contribution reaches the
+ * length-normalised tolerance tau / L_q.  Source: "MassAlloc Attention: Let Attention
+ * Allocate Its Own Compute" (§2.1 tolerance, §2.2 Eq. (3) online forward test and
+ * Eq. (4) offline backward test, §2.4 split-KV decoding, App. A Algorithms 1 and 2).
+ *
+ * Conventions shared by every entry point
+ *   - All tensor pointers are caller-owned DEVICE memory, contiguous, 16-byte aligned.
+ *   - Layouts: Q, O, dO, dQ [B, L, H, d]; K, V, dK, dV [B, L, H_kv, d];
+ *     LSE [B, H, L] float32, natural-log log-sum-exp of the scaled scores over the
+ *     retained keys (the page's final l = m + log l).  Query head h reads KV head
+ *     h / (H / H_kv) (grouped-query attention).
+ *   - Scores are s = scale * <q, k>; tiles are 128 query rows x 128 keys; tile (i, j)
+ *     is query block i, key block j.  The forward visits j = i, i-1, ..., 0 (diagonal
+ *     first) and skips a tile only when every valid row with a legal key in it has
+ *     max_k s - log Z_q < log(tau / L_q), L_q = q + 1 (strict; ties retain).
+ *   - tau >= 0.  tau == 0 means "never skip" and runs the same library's dense
+ *     FlashAttention-style kernels; MALA_FLAG_ALWAYS_TEST runs the retention test
+ *     anyway (it then retains everything) to measure its overhead.
+ *   - dtype: MALA_BF16 (tensor-core path; d in {64, 128}) or MALA_FP32 (fp32 SIMT path
+ *     for small problems; d <= 128).
+ *   - tile_mask (optional, may be NULL): debug output of the decisions, one byte per
+ *     legal tile, 1 = retained, 0 = skipped.  Forward / backward: [B, H, T, T] with
+ *     T = ceil(L / 128), entry [b][h][i][j]; decode: [B, H, T] with T = ceil(N_k / 128).
+ *     Entries of illegal tiles (j > i) are left untouched.  The method itself never
+ *     materialises a mask; this buffer exists only for testing and statistics.
+ *   - workspace: caller-provided device scratch of at least the size returned by the
+ *     matching *_workspace_bytes query.  Passing workspace == NULL makes the library
+ *     allocate it stream-ordered (cudaMallocAsync / cudaFreeAsync) on `stream`.  The
+ *     first 256 bytes of any workspace hold counters and the device error word.
+ *   - stream: a cudaStream_t (NULL = legacy default stream).  All work is enqueued
+ *     asynchronously; no entry point synchronises the host.
+ *   - Errors: arguments are validated before anything is launched
+ *     (MALA_ERR_INVALID_ARG / MALA_ERR_UNSUPPORTED); launch failures return
+ *     MALA_ERR_CUDA.  A kernel whose internal wait runs out of its time budget records
+ *     MALA_ERR_TIMEOUT in the workspace error word and returns early instead of
+ *     hanging; read it with mala_read_device_error().
+ */
+#ifndef MALA_H
+#define MALA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MALA_OK = 0,
+  MALA_ERR_INVALID_ARG = 1,
+  MALA_ERR_UNSUPPORTED = 2,
+  MALA_ERR_CUDA = 3,
+  MALA_ERR_TIMEOUT = 4,
+  MALA_ERR_WORKSPACE = 5
+} mala_status;
+
+typedef enum { MALA_BF16 = 0, MALA_FP32 = 1 } mala_dtype;
+
+/* flags */
+#define MALA_FLAG_ALWAYS_TEST 1u /* evaluate the retention test even when tau == 0 */
+
+/*
+ * mala_fwd - MALA forward (training forward and inference prefill).
+ * "MassAlloc Attention", §2.2 (online sparse softmax, Eq. (1)-(3)), App. A Algorithm 1
+ * and A.1 (fused forward execution).
+ *   Q [B,L,H,d], K/V [B,L,H_kv,d] in, O [B,L,H,d] out (same dtype as the inputs),
+ *   LSE [B,H,L] float32 out.  Causal, N_q = N_k = L >= 1.
+ */
+mala_status mala_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE, int B,
+                     int H, int H_kv, int L, int d, int dtype, float scale, float tau,
+                     unsigned flags, void* workspace, size_t workspace_bytes,
+                     uint8_t* tile_mask, void* stream);
+
+/*
+ * mala_bwd - MALA backward.
+ * "MassAlloc Attention", §2.2 (offline sparse probability, Eq. (4)), App. A
+ * Algorithm 2 and A.1 (fused backward execution).  O and LSE are the forward's
+ * outputs; D = rowsum(O * dO) is formed inside.  dQ, dK, dV are fully written (not
+ * accumulated); dK / dV sum the contributions of the H / H_kv query heads of each KV
+ * head.  The workspace holds a float32 dQ accumulator [B,L,H,d] and D [B,H,L].
+ */
+mala_status mala_bwd(const void* Q, const void* K, const void* V, const void* O,
+                     const float* LSE, const void* dO, void* dQ, void* dK, void* dV, int B,
+                     int H, int H_kv, int L, int d, int dtype, float scale, float tau,
+                     unsigned flags, void* workspace, size_t workspace_bytes,
+                     uint8_t* tile_mask, void* stream);
+
+/*
+ * mala_decode - MALA split-KV decoding of one query token per sequence.
+ * "MassAlloc Attention", §2.1 (L_0 = N_k, including the current token), §2.4 and A.1
+ * (each split tests against its own partial normaliser; splits merged by the
+ * normaliser-aware log-sum-exp reduction).
+ *   q [B,H,d]; Kc, Vc [B,N_k,H_kv,d] (the cache already holds the current token at
+ *   position N_k - 1); O [B,H,d] out; LSE [B,H] float32 out.
+ *   Key tiles of 128; split s of S owns tiles [s*T/S, (s+1)*T/S) (integer division)
+ *   and visits them newest first.  num_splits = 0 picks mala_decode_num_splits().
+ *   The retained support depends on the split count (the page says so).
+ */
+mala_status mala_decode(const void* q, const void* Kc, const void* Vc, void* O, float* LSE,
+                        int B, int H, int H_kv, int Nk, int d, int dtype, float scale,
+                        float tau, int num_splits, unsigned flags, void* workspace,
+                        size_t workspace_bytes, uint8_t* tile_mask, void* stream);
+
+/* Workspace sizes (bytes) for the calls above; 0 on invalid arguments. */
+size_t mala_fwd_workspace_bytes(int B, int H, int H_kv, int L, int d, int dtype);
+size_t mala_bwd_workspace_bytes(int B, int H, int H_kv, int L, int d, int dtype);
+size_t mala_decode_workspace_bytes(int B, int H, int H_kv, int Nk, int d, int dtype,
+                                   int num_splits);
+
+/* The split count used when mala_decode is given num_splits = 0 (deterministic). */
+int mala_decode_num_splits(int B, int H, int H_kv, int Nk);
+
+/* Reads the device error word of a workspace (synchronises `stream`).  *out receives
+ * 0 or a mala_status code in its low byte (upper bits: which wait gave up).  Clears
+ * the word when clear != 0. */
+mala_status mala_read_device_error(const void* workspace, void* stream, uint32_t* out,
+                                   int clear);
+
+/* Sets the wall-clock budget of every internal wait (default 2 s; test hook). */
+mala_status mala_set_wait_budget_ns(uint64_t ns);
+
+const char* mala_status_string(mala_status s);
+
+/* Library version, e.g. 100 = 0.1.0. */
+int mala_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MALA_H */

@@ -1,0 +1,262 @@
+// C-ABI entry points of the MALA library: argument validation, TMA descriptor
+// construction, workspace handling and kernel launches.  See include/mala.h.
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "mala.h"
+#include "mala_common.cuh"
+
+namespace mala {
+cudaError_t launch_fwd_bf16(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                            const FwdParams& p, int d, bool screen, int grid, cudaStream_t stream);
+mala_status bwd_dispatch(const void* Q, const void* K, const void* V, const void* O,
+                         const float* LSE, const void* dO, void* dQ, void* dK, void* dV, int B,
+                         int H, int Hkv, int L, int d, int dtype, float scale, float tau,
+                         unsigned flags, uint8_t* ws, uint8_t* tile_mask, uint64_t budget_ns,
+                         cudaStream_t stream);
+size_t bwd_workspace_bytes(int B, int H, int Hkv, int L, int d, int dtype);
+mala_status decode_dispatch(const void* q, const void* K, const void* V, void* O, float* LSE,
+                            int B, int H, int Hkv, int Nk, int d, int dtype, float scale,
+                            float tau, int num_splits, unsigned flags, uint8_t* ws,
+                            uint8_t* tile_mask, uint64_t budget_ns, cudaStream_t stream);
+size_t decode_workspace_bytes(int B, int H, int Hkv, int Nk, int d, int dtype, int num_splits);
+int decode_auto_splits(int B, int Hkv, int Nk);
+mala_status fp32_fwd(const float* Q, const float* K, const float* V, float* O, float* LSE, int B,
+                     int H, int Hkv, int L, int d, float scale, float tau, bool screen,
+                     uint8_t* tile_mask, cudaStream_t stream);
+
+// ---------------------------------------------------------------------------- shared host helpers
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(f);
+  });
+  return fn;
+}
+
+// 4-D bf16 tensor [n3][n2][n1][n0] (n0 fastest), box {64, 1, 128, 1}, 128-byte swizzle.
+bool make_tile_map(CUtensorMap* m, const void* base, int n0, int n1, int n2, int n3) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[4] = {(cuuint64_t)n0, (cuuint64_t)n1, (cuuint64_t)n2, (cuuint64_t)n3};
+  cuuint64_t strides[3] = {(cuuint64_t)n0 * 2, (cuuint64_t)n0 * n1 * 2,
+                           (cuuint64_t)n0 * n1 * n2 * 2};
+  cuuint32_t box[4] = {64, 1, 128, 1};
+  cuuint32_t es[4] = {1, 1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box,
+             es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 148;
+  return n > 0 ? n : 148;
+}
+
+static uint64_t g_budget_ns = 2000000000ull;
+
+uint64_t wait_budget_ns() { return g_budget_ns; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool common_args_ok(int B, int H, int Hkv, int L, int d, int dtype, float scale, float tau) {
+  if (B <= 0 || H <= 0 || Hkv <= 0 || L <= 0 || d <= 0) return false;
+  if (H % Hkv != 0) return false;
+  if (!(std::isfinite(scale) && scale > 0.f)) return false;
+  if (!(std::isfinite(tau) && tau >= 0.f)) return false;
+  if (dtype != MALA_BF16 && dtype != MALA_FP32) return false;
+  return true;
+}
+
+// Runs `body(ws)` with either the caller's workspace or a stream-ordered allocation.
+template <class F>
+mala_status with_workspace(void* workspace, size_t ws_bytes, size_t need, cudaStream_t stream,
+                           F body) {
+  if (workspace) {
+    if (ws_bytes < need) return MALA_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return MALA_ERR_INVALID_ARG;
+    return body(static_cast<uint8_t*>(workspace));
+  }
+  void* ws = nullptr;
+  if (cudaMallocAsync(&ws, need, stream) != cudaSuccess) return MALA_ERR_CUDA;
+  if (cudaMemsetAsync(ws, 0, kWorkspaceHeader, stream) != cudaSuccess) {
+    cudaFreeAsync(ws, stream);
+    return MALA_ERR_CUDA;
+  }
+  mala_status st = body(static_cast<uint8_t*>(ws));
+  if (cudaFreeAsync(ws, stream) != cudaSuccess && st == MALA_OK) st = MALA_ERR_CUDA;
+  return st;
+}
+
+}  // namespace mala
+
+using namespace mala;
+
+extern "C" {
+
+int mala_version(void) { return 100; }
+
+const char* mala_status_string(mala_status s) {
+  switch (s) {
+    case MALA_OK: return "ok";
+    case MALA_ERR_INVALID_ARG: return "invalid argument";
+    case MALA_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+    case MALA_ERR_CUDA: return "CUDA error";
+    case MALA_ERR_TIMEOUT: return "device wait timed out";
+    case MALA_ERR_WORKSPACE: return "workspace too small";
+  }
+  return "unknown status";
+}
+
+mala_status mala_set_wait_budget_ns(uint64_t ns) {
+  if (ns == 0) return MALA_ERR_INVALID_ARG;
+  g_budget_ns = ns;
+  return MALA_OK;
+}
+
+mala_status mala_read_device_error(const void* workspace, void* stream, uint32_t* out,
+                                   int clear) {
+  if (!workspace || !out) return MALA_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint32_t v = 0;
+  if (cudaMemcpyAsync(&v, workspace, 4, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return MALA_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return MALA_ERR_CUDA;
+  *out = v;
+  if (clear && cudaMemsetAsync(const_cast<void*>(workspace), 0, 4, s) != cudaSuccess)
+    return MALA_ERR_CUDA;
+  return MALA_OK;
+}
+
+size_t mala_fwd_workspace_bytes(int B, int H, int H_kv, int L, int d, int dtype) {
+  if (!common_args_ok(B, H, H_kv, L, d, dtype, 1.f, 0.f)) return 0;
+  return kWorkspaceHeader;
+}
+
+mala_status mala_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE, int B,
+                     int H, int H_kv, int L, int d, int dtype, float scale, float tau,
+                     unsigned flags, void* workspace, size_t workspace_bytes,
+                     uint8_t* tile_mask, void* stream) {
+  if (!common_args_ok(B, H, H_kv, L, d, dtype, scale, tau)) return MALA_ERR_INVALID_ARG;
+  if (!Q || !K || !V || !O || !LSE) return MALA_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O))
+    return MALA_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const bool screen = (tau > 0.f) || (flags & MALA_FLAG_ALWAYS_TEST);
+  const int T = (L + kTile - 1) / kTile;
+  if (dtype == MALA_FP32) {
+    if (d > 128) return MALA_ERR_UNSUPPORTED;
+    return fp32_fwd(static_cast<const float*>(Q), static_cast<const float*>(K),
+                    static_cast<const float*>(V), static_cast<float*>(O), LSE, B, H, H_kv, L, d,
+                    scale, tau, screen, tile_mask, st);
+  }
+  if (d != 64 && d != 128) return MALA_ERR_UNSUPPORTED;
+  if ((long long)B * L > (1ll << 31) || (long long)B * H * T > (1ll << 30))
+    return MALA_ERR_UNSUPPORTED;
+  CUtensorMap tq, tk, tv;
+  if (!make_tile_map(&tq, Q, d, H, L, B) || !make_tile_map(&tk, K, d, H_kv, L, B) ||
+      !make_tile_map(&tv, V, d, H_kv, L, B))
+    return MALA_ERR_CUDA;
+  const size_t need = mala_fwd_workspace_bytes(B, H, H_kv, L, d, dtype);
+  return with_workspace(workspace, workspace_bytes, need, st, [&](uint8_t* ws) -> mala_status {
+    uint32_t* hdr = reinterpret_cast<uint32_t*>(ws);
+    if (cudaMemsetAsync(hdr + kHdrSched0, 0, 3 * sizeof(uint32_t), st) != cudaSuccess)
+      return MALA_ERR_CUDA;
+    FwdParams p;
+    p.B = B; p.H = H; p.Hkv = H_kv; p.L = L; p.T = T; p.G = H / H_kv;
+    p.npairs = (p.G + 1) / 2;
+    p.n_units = T * B * H_kv * p.npairs;
+    p.scale_log2 = scale * kLog2e;
+    p.log2_tau = (tau > 0.f) ? std::log2(tau) : -INFINITY;
+    p.O = O; p.LSE = LSE; p.tile_mask = tile_mask;
+    p.err = hdr + kHdrError;
+    p.sched = hdr + kHdrSched0;
+    p.budget_ns = wait_budget_ns();
+    const int grid = p.n_units < sm_count() ? p.n_units : sm_count();
+    cudaError_t e = launch_fwd_bf16(tq, tk, tv, p, d, screen, grid, st);
+    return e == cudaSuccess ? MALA_OK : MALA_ERR_CUDA;
+  });
+}
+
+size_t mala_bwd_workspace_bytes(int B, int H, int H_kv, int L, int d, int dtype) {
+  if (!common_args_ok(B, H, H_kv, L, d, dtype, 1.f, 0.f)) return 0;
+  return bwd_workspace_bytes(B, H, H_kv, L, d, dtype);
+}
+
+mala_status mala_bwd(const void* Q, const void* K, const void* V, const void* O,
+                     const float* LSE, const void* dO, void* dQ, void* dK, void* dV, int B,
+                     int H, int H_kv, int L, int d, int dtype, float scale, float tau,
+                     unsigned flags, void* workspace, size_t workspace_bytes,
+                     uint8_t* tile_mask, void* stream) {
+  if (!common_args_ok(B, H, H_kv, L, d, dtype, scale, tau)) return MALA_ERR_INVALID_ARG;
+  if (!Q || !K || !V || !O || !LSE || !dO || !dQ || !dK || !dV) return MALA_ERR_INVALID_ARG;
+  for (const void* ptr : {Q, K, V, O, dO, static_cast<const void*>(dQ),
+                          static_cast<const void*>(dK), static_cast<const void*>(dV)})
+    if (!aligned16(ptr)) return MALA_ERR_INVALID_ARG;
+  if (dtype == MALA_BF16 && d != 64 && d != 128) return MALA_ERR_UNSUPPORTED;
+  if (dtype == MALA_FP32 && d > 128) return MALA_ERR_UNSUPPORTED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t need = bwd_workspace_bytes(B, H, H_kv, L, d, dtype);
+  return with_workspace(workspace, workspace_bytes, need, st, [&](uint8_t* ws) -> mala_status {
+    return bwd_dispatch(Q, K, V, O, LSE, dO, dQ, dK, dV, B, H, H_kv, L, d, dtype, scale, tau,
+                        flags, ws, tile_mask, wait_budget_ns(), st);
+  });
+}
+
+int mala_decode_num_splits(int B, int H, int H_kv, int Nk) {
+  if (B <= 0 || H <= 0 || H_kv <= 0 || Nk <= 0 || H % H_kv) return 0;
+  return decode_auto_splits(B, H_kv, Nk);
+}
+
+size_t mala_decode_workspace_bytes(int B, int H, int H_kv, int Nk, int d, int dtype,
+                                   int num_splits) {
+  if (!common_args_ok(B, H, H_kv, Nk, d, dtype, 1.f, 0.f)) return 0;
+  if (num_splits == 0) num_splits = decode_auto_splits(B, H_kv, Nk);
+  const int T = (Nk + kTile - 1) / kTile;
+  if (num_splits < 1 || num_splits > T) return 0;
+  return decode_workspace_bytes(B, H, H_kv, Nk, d, dtype, num_splits);
+}
+
+mala_status mala_decode(const void* q, const void* Kc, const void* Vc, void* O, float* LSE,
+                        int B, int H, int H_kv, int Nk, int d, int dtype, float scale,
+                        float tau, int num_splits, unsigned flags, void* workspace,
+                        size_t workspace_bytes, uint8_t* tile_mask, void* stream) {
+  if (!common_args_ok(B, H, H_kv, Nk, d, dtype, scale, tau)) return MALA_ERR_INVALID_ARG;
+  if (!q || !Kc || !Vc || !O || !LSE) return MALA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(Kc) || !aligned16(Vc) || !aligned16(O))
+    return MALA_ERR_INVALID_ARG;
+  const int T = (Nk + kTile - 1) / kTile;
+  if (num_splits == 0) num_splits = decode_auto_splits(B, H_kv, Nk);
+  if (num_splits < 1 || num_splits > T) return MALA_ERR_INVALID_ARG;
+  if (dtype == MALA_BF16 && d != 64 && d != 128) return MALA_ERR_UNSUPPORTED;
+  if (dtype == MALA_FP32 && d > 128) return MALA_ERR_UNSUPPORTED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t need = decode_workspace_bytes(B, H, H_kv, Nk, d, dtype, num_splits);
+  return with_workspace(workspace, workspace_bytes, need, st, [&](uint8_t* ws) -> mala_status {
+    return decode_dispatch(q, Kc, Vc, O, LSE, B, H, H_kv, Nk, d, dtype, scale, tau, num_splits,
+                           flags, ws, tile_mask, wait_budget_ns(), st);
+  });
+}
+
+}  // extern "C"

@@ -1,0 +1,9 @@
+// fp32 SIMT path (placeholder).
+#include <cuda_runtime.h>
+#include "mala.h"
+namespace mala {
+mala_status fp32_fwd(const float*, const float*, const float*, float*, float*, int, int, int, int,
+                     int, float, float, bool, uint8_t*, cudaStream_t) {
+  return MALA_ERR_UNSUPPORTED;
+}
+}  // namespace mala

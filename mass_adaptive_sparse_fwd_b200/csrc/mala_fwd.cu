@@ -1,0 +1,459 @@
+// MALA forward kernel for sm_100a (bf16, head dim 64 or 128).
+//
+// "MassAlloc Attention: Let Attention Allocate Its Own Compute", §2.2 (online sparse
+// softmax, Eq. (1)-(3)), App. A Algorithm 1 and A.1 (fused forward execution).
+//
+// One persistent CTA per SM pulls work units from an atomic counter.  A unit is one
+// 128-row query block i of two query heads that share a KV head (two "slots"), so both
+// slots stream the same K_j / V_j tiles; units are numbered heaviest first (largest i).
+// Within a unit the key blocks are visited j = i, i-1, ..., 0 (diagonal first).
+//
+// Warp roles (384 threads):
+//   warp 0      TMA producer: Q of both slots, then K_j and V_j per key block into a
+//               ring of NS stages.  V is fetched together with K (see below).
+//   warp 1      TMEM owner and UMMA issuer: S_s = Q_s K_j^T (SS, both K-major) into
+//               TMEM, and O_s += P_s V_j (TS: P in TMEM, V MN-major) for retained tiles.
+//   warps 4-7   softmax / retention test for slot 0 (thread = query row = TMEM lane)
+//   warps 8-11  same for slot 1
+// TMEM columns: S_0 [0,128), S_1 [128,256), O_0 [256,256+D), O_1 [256+D, 256+2D).
+// P_s (bf16, packed in pairs) overwrites the first 64 columns of S_s.
+//
+// Retention test (Eq. 3) per row q in the log2 domain: with the running state
+// (m, l) of retained tiles, log2 Z = m + log2 l.  A row keeps the tile if l == 0
+// (its first legal tile) or rowmax(S) * scale * log2(e) >= m + log2(l) + log2(tau/L_q),
+// L_q = q + 1; rows with no legal key in the tile (above the diagonal, or q >= L) do
+// not vote.  The tile is retained if any row keeps it (bar.red.or over the 128
+// threads).  A skipped tile leaves m, l and O untouched and costs only the QK^T MMA,
+// the TMEM load of S and the row maxima: no exponentials, no P store, no PV MMA.
+//
+// The running max used for P is updated lazily (only when a row max exceeds it by
+// more than 8 in log2 units), so O is rescaled in TMEM only on such jumps; log Z is
+// m + log2 l for any m, so the test is unaffected.
+//
+// V loading: K_j and V_j are fetched together, before the decision for tile j exists.
+// The forward is tensor-core bound and deciding first would put the V latency on the
+// critical path of every retained tile; the skipped work is the exponentials and the
+// PV MMA.  (Decode, which is bandwidth bound, gates its V loads on the decision.)
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+
+#include "mala_common.cuh"
+#include "sm100.cuh"
+
+namespace mala {
+
+namespace {
+
+template <int D>
+struct FwdCfg {
+  static constexpr int NS = (D == 128) ? 2 : 4;          // K/V ring stages (K and V tiles each)
+  static constexpr int TILE_BYTES = kTile * D * 2;       // one 128 x D bf16 tile
+  static constexpr int BOXES = D / 64;                   // 64-column TMA boxes per tile
+  static constexpr int SMEM = 2 * TILE_BYTES + 2 * NS * TILE_BYTES + 1024;
+  static constexpr int THREADS = 384;
+};
+
+struct FwdShared {
+  uint64_t q_full[2], q_empty[2];
+  uint64_t k_full[4], v_full[4], kv_empty[4];
+  uint64_t s_full[2], p_full[2], o_done[2];
+  uint64_t sched_full[2], sched_empty[2];
+  uint64_t final_bar;
+  int sched_ring[2];
+  uint32_t dec[2];
+  uint32_t tmem_base;
+  uint32_t abort_flag;
+};
+
+struct Unit {
+  int b, g, i, h0;
+  bool active[2];
+};
+
+__device__ __forceinline__ Unit decode_unit(const FwdParams& p, int u) {
+  const int nbg = p.B * p.Hkv * p.npairs;
+  Unit w;
+  w.i = p.T - 1 - u / nbg;
+  const int r = u % nbg;
+  w.b = r / (p.Hkv * p.npairs);
+  w.g = (r / p.npairs) % p.Hkv;
+  const int hp = r % p.npairs;
+  w.h0 = w.g * p.G + 2 * hp;
+  w.active[0] = true;
+  w.active[1] = (2 * hp + 1) < p.G;
+  return w;
+}
+
+template <int D, bool kScreen>
+__global__ void __launch_bounds__(384, 1)
+    mala_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                    const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
+  using C = FwdCfg<D>;
+  constexpr int NS = C::NS;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* sQ = smem;                                  // 2 tiles
+  uint8_t* sK = smem + 2 * C::TILE_BYTES;              // NS tiles
+  uint8_t* sV = sK + NS * C::TILE_BYTES;               // NS tiles
+  __shared__ FwdShared sh;
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+
+  if (tid == 0) {
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&sh.q_full[s], 1);
+      mbar_init(&sh.q_empty[s], 1);
+      mbar_init(&sh.s_full[s], 1);
+      mbar_init(&sh.p_full[s], 128);
+      mbar_init(&sh.o_done[s], 1);
+      mbar_init(&sh.sched_full[s], 1);
+      mbar_init(&sh.sched_empty[s], 1 + 256);
+    }
+    for (int st = 0; st < NS; ++st) {
+      mbar_init(&sh.k_full[st], 1);
+      mbar_init(&sh.v_full[st], 1);
+      mbar_init(&sh.kv_empty[st], 1);
+    }
+    mbar_init(&sh.final_bar, 1);
+    sh.abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&sh.tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tb = sh.tmem_base;
+  const AbortState ast{&sh.abort_flag, p.err, p.budget_ns, 0x100u};
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      uint32_t c = 0;                  // K/V tiles issued (all units)
+      uint32_t nq[2] = {0, 0};         // Q loads issued per slot
+      int last_q_stage_used = 0;
+      (void)last_q_stage_used;
+      bool ok = true;
+      for (uint32_t k = 0; ok; ++k) {
+        const int ring = k & 1;
+        if (k >= 2 && !(ok = mbar_wait(&sh.sched_empty[ring], ((k >> 1) - 1) & 1, ast, 1))) break;
+        const int u = static_cast<int>(atomicAdd(p.sched, 1u));
+        sh.sched_ring[ring] = u;
+        mbar_arrive(&sh.sched_full[ring]);
+        if (u >= p.n_units) break;
+        const Unit w = decode_unit(p, u);
+        for (int s = 0; s < 2 && ok; ++s) {
+          if (!w.active[s]) continue;
+          if (nq[s] > 0 && !(ok = mbar_wait(&sh.q_empty[s], (nq[s] - 1) & 1, ast, 2))) break;
+          mbar_arrive_expect_tx(&sh.q_full[s], C::TILE_BYTES);
+          for (int x = 0; x < C::BOXES; ++x)
+            tma_load_4d(sQ + s * C::TILE_BYTES + x * 16384, &tmQ, &sh.q_full[s], x * 64,
+                        w.h0 + s, w.i * kTile, w.b);
+          ++nq[s];
+        }
+        for (int t = 0; t <= w.i && ok; ++t, ++c) {
+          const int j = w.i - t;
+          const int st = c % NS;
+          if (c >= NS && !(ok = mbar_wait(&sh.kv_empty[st], ((c / NS) - 1) & 1, ast, 3))) break;
+          mbar_arrive_expect_tx(&sh.k_full[st], C::TILE_BYTES);
+          for (int x = 0; x < C::BOXES; ++x)
+            tma_load_4d(sK + st * C::TILE_BYTES + x * 16384, &tmK, &sh.k_full[st], x * 64, w.g,
+                        j * kTile, w.b);
+          mbar_arrive_expect_tx(&sh.v_full[st], C::TILE_BYTES);
+          for (int x = 0; x < C::BOXES; ++x)
+            tma_load_4d(sV + st * C::TILE_BYTES + x * 16384, &tmV, &sh.v_full[st], x * 64, w.g,
+                        j * kTile, w.b);
+        }
+      }
+      if (!ok) {
+        // drain: wait (bounded) for the loads this CTA still has in flight
+        AbortState drain = ast;
+        uint32_t zero = 0;
+        drain.flag = &zero;
+        drain.budget_ns = 200000000ull;
+        for (uint32_t cc = (c > NS ? c - NS : 0); cc < c; ++cc) {
+          mbar_wait(&sh.k_full[cc % NS], (cc / NS) & 1, drain, 4);
+          mbar_wait(&sh.v_full[cc % NS], (cc / NS) & 1, drain, 4);
+        }
+        for (int s = 0; s < 2; ++s)
+          if (nq[s] > 0) mbar_wait(&sh.q_full[s], (nq[s] - 1) & 1, drain, 4);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t id_qk = idesc_bf16(128, 128, 0, 0);
+      constexpr uint32_t id_pv = idesc_bf16(128, D, 0, 1);
+      uint32_t c = 0;
+      uint32_t nq[2] = {0, 0};
+      uint32_t np[2] = {0, 0};  // p_full phases consumed per slot
+      bool ok = true;
+      auto issue_qk = [&](int s, int st) {
+        const uint32_t qa = smem_u32(sQ + s * C::TILE_BYTES);
+        const uint32_t ka = smem_u32(sK + st * C::TILE_BYTES);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+          umma_ss(tb + s * 128, sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(ka + off, 16, 1024),
+                  id_qk, kk > 0);
+        }
+        umma_commit(&sh.s_full[s]);
+      };
+      for (uint32_t k = 0; ok; ++k) {
+        const int ring = k & 1;
+        if (!(ok = mbar_wait(&sh.sched_full[ring], (k >> 1) & 1, ast, 10))) break;
+        const int u = sh.sched_ring[ring];
+        mbar_arrive(&sh.sched_empty[ring]);
+        if (u >= p.n_units) break;
+        const Unit w = decode_unit(p, u);
+        for (int s = 0; s < 2 && ok; ++s) {
+          if (!w.active[s]) continue;
+          ok = mbar_wait(&sh.q_full[s], nq[s] & 1, ast, 11);
+          ++nq[s];
+        }
+        if (!ok) break;
+        bool o_started[2] = {false, false};
+        const int n = w.i + 1;
+        // prologue: S for the diagonal tile
+        {
+          const int st = c % NS;
+          if (!(ok = mbar_wait(&sh.k_full[st], (c / NS) & 1, ast, 12))) break;
+          tc_fence_after();
+          for (int s = 0; s < 2; ++s)
+            if (w.active[s]) issue_qk(s, st);
+        }
+        for (int t = 0; t < n && ok; ++t, ++c) {
+          const int st = c % NS;
+          bool v_ready = false, k_next_ready = false;
+          for (int s = 0; s < 2 && ok; ++s) {
+            if (!w.active[s]) continue;
+            if (!(ok = mbar_wait(&sh.p_full[s], np[s] & 1, ast, 13))) break;
+            ++np[s];
+            tc_fence_after();
+            if (sh.dec[s]) {
+              if (!v_ready && !(ok = v_ready = mbar_wait(&sh.v_full[st], (c / NS) & 1, ast, 14)))
+                break;
+              const uint32_t va = smem_u32(sV + st * C::TILE_BYTES);
+#pragma unroll
+              for (int kk = 0; kk < 8; ++kk)
+                umma_ts(tb + 256 + s * D, tb + s * 128 + kk * 8,
+                        sdesc_sw128(va + kk * 2048, 16384, 1024), id_pv,
+                        (o_started[s] || kk > 0) ? 1u : 0u);
+              o_started[s] = true;
+              umma_commit(&sh.o_done[s]);
+            }
+            if (t + 1 < n) {
+              const uint32_t c1 = c + 1;
+              if (!k_next_ready &&
+                  !(ok = k_next_ready = mbar_wait(&sh.k_full[c1 % NS], (c1 / NS) & 1, ast, 15)))
+                break;
+              tc_fence_after();
+              issue_qk(s, c1 % NS);
+            }
+          }
+          if (!ok) break;
+          // the stage is released only after its V load landed, even if no slot used it
+          if (!v_ready && !(ok = mbar_wait(&sh.v_full[st], (c / NS) & 1, ast, 16))) break;
+          umma_commit(&sh.kv_empty[st]);
+        }
+        if (!ok) break;
+        for (int s = 0; s < 2; ++s)
+          if (w.active[s]) umma_commit(&sh.q_empty[s]);
+      }
+      // wait for every MMA this thread issued before TMEM is released
+      umma_commit(&sh.final_bar);
+      AbortState fin = ast;
+      uint32_t zero = 0;
+      fin.flag = &zero;
+      mbar_wait(&sh.final_bar, 0, fin, 17);
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------------ softmax
+    const int s = (warp - 4) >> 2;          // slot
+    const int wq = warp & 3;                // TMEM lane quarter
+    const int r = wq * 32 + lane;           // row within the tile
+    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+    const uint32_t tS = tb + s * 128 + lane_off;
+    const uint32_t tO = tb + 256 + s * D + lane_off;
+    const float NEG_INF = -INFINITY;
+    uint32_t ns = 0, npv = 0;
+    bool ok = true;
+    for (uint32_t k = 0; ok; ++k) {
+      const int ring = k & 1;
+      if (!(ok = mbar_wait(&sh.sched_full[ring], (k >> 1) & 1, ast, 20))) break;
+      const int u = sh.sched_ring[ring];
+      mbar_arrive(&sh.sched_empty[ring]);
+      if (u >= p.n_units) break;
+      const Unit w = decode_unit(p, u);
+      if (!w.active[s]) continue;
+      const int h = w.h0 + s;
+      const int q = w.i * kTile + r;
+      const bool valid = q < p.L;
+      const float thr2 = kScreen ? (p.log2_tau - __log2f(static_cast<float>(q + 1))) : NEG_INF;
+      float m2 = NEG_INF, l = 0.f;
+      const uint32_t npv_unit0 = npv;
+      const int n = w.i + 1;
+      for (int t = 0; t < n; ++t) {
+        const int j = w.i - t;
+        if (!(ok = mbar_wait(&sh.s_full[s], ns & 1, ast, 21))) break;
+        ++ns;
+        tc_fence_after();
+        uint32_t v[4][32];
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) tmem_ld32(tS + cc * 32, v[cc]);
+        tmem_wait_ld();
+        float rmax = NEG_INF;
+        if (t == 0 || !valid) {
+          const int lim = valid ? r : -1;  // diagonal tile: keys c <= r are legal
+#pragma unroll
+          for (int cc = 0; cc < 4; ++cc)
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              float x = __uint_as_float(v[cc][e]) * p.scale_log2;
+              x = (cc * 32 + e <= lim) ? x : NEG_INF;
+              v[cc][e] = __float_as_uint(x);
+              rmax = fmaxf(rmax, x);
+            }
+        } else {
+#pragma unroll
+          for (int cc = 0; cc < 4; ++cc)
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              const float x = __uint_as_float(v[cc][e]) * p.scale_log2;
+              v[cc][e] = __float_as_uint(x);
+              rmax = fmaxf(rmax, x);
+            }
+        }
+        bool keep = true;
+        if (kScreen) {
+          const bool mine = (rmax != NEG_INF) && (l == 0.f || rmax >= m2 + __log2f(l) + thr2);
+          keep = named_bar_or(1 + s, 128, mine);
+        }
+        if (p.tile_mask && r == 0)
+          p.tile_mask[((static_cast<size_t>(w.b) * p.H + h) * p.T + w.i) * p.T + j] = keep ? 1 : 0;
+        if (!keep) {
+          if (r == 0) sh.dec[s] = 0;
+          tc_fence_before();
+          mbar_arrive(&sh.p_full[s]);
+          continue;
+        }
+        // lazy running-max update
+        float m_new = m2;
+        bool rescale = false;
+        if (rmax > m2 + 8.0f) {
+          m_new = rmax;
+          rescale = (l > 0.f);
+        }
+        const float m_use = (m_new == NEG_INF) ? 0.f : m_new;
+        const float alpha = rescale ? fast_exp2(m2 - m_new) : 1.f;
+        if (__any_sync(0xffffffffu, rescale)) {
+          // the previous PV of this slot must have landed before O is touched
+          if (!(ok = mbar_wait(&sh.o_done[s], (npv - 1) & 1, ast, 22))) break;
+          tc_fence_after();
+#pragma unroll
+          for (int cc = 0; cc < D / 32; ++cc) {
+            uint32_t o[32];
+            tmem_ld32(tO + cc * 32, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            tmem_st32(tO + cc * 32, o);
+          }
+        }
+        float psum = 0.f;
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const float p0 = fast_exp2(__uint_as_float(v[cc][2 * e]) - m_use);
+            const float p1 = fast_exp2(__uint_as_float(v[cc][2 * e + 1]) - m_use);
+            psum += p0 + p1;
+            pk[e] = pack_bf16(p0, p1);
+          }
+          tmem_st16(tS + cc * 16, pk);
+        }
+        tmem_wait_st();
+        l = l * alpha + psum;
+        m2 = m_new;
+        if (r == 0) sh.dec[s] = 1;
+        tc_fence_before();
+        mbar_arrive(&sh.p_full[s]);
+        ++npv;
+      }
+      if (!ok) break;
+      // epilogue: O = acc / l, LSE = (m + log2 l) * ln 2
+      if (npv > npv_unit0) {
+        if (!(ok = mbar_wait(&sh.o_done[s], (npv - 1) & 1, ast, 23))) break;
+      }
+      tc_fence_after();
+      const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
+      __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.O) +
+                            ((static_cast<size_t>(w.b) * p.L + q) * p.H + h) * D;
+#pragma unroll
+      for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t o[32];
+        tmem_ld32(tO + cc * 32, o);
+        tmem_wait_ld();
+        if (valid) {
+#pragma unroll
+          for (int e8 = 0; e8 < 4; ++e8) {
+            uint4 pk;
+            pk.x = pack_bf16(__uint_as_float(o[e8 * 8 + 0]) * inv_l, __uint_as_float(o[e8 * 8 + 1]) * inv_l);
+            pk.y = pack_bf16(__uint_as_float(o[e8 * 8 + 2]) * inv_l, __uint_as_float(o[e8 * 8 + 3]) * inv_l);
+            pk.z = pack_bf16(__uint_as_float(o[e8 * 8 + 4]) * inv_l, __uint_as_float(o[e8 * 8 + 5]) * inv_l);
+            pk.w = pack_bf16(__uint_as_float(o[e8 * 8 + 6]) * inv_l, __uint_as_float(o[e8 * 8 + 7]) * inv_l);
+            *reinterpret_cast<uint4*>(orow + cc * 32 + e8 * 8) = pk;
+          }
+        }
+      }
+      if (valid) p.LSE[(static_cast<size_t>(w.b) * p.H + h) * p.L + q] = (m2 + __log2f(l)) * kLn2;
+      tc_fence_before();
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tb, 512);
+}
+
+}  // namespace
+
+// ---------------------------------------------------------------------------- launch
+
+template <int D, bool kScreen>
+static cudaError_t launch_fwd_impl(const CUtensorMap& tq, const CUtensorMap& tk,
+                                   const CUtensorMap& tv, const FwdParams& p, int grid,
+                                   cudaStream_t stream) {
+  using C = FwdCfg<D>;
+  auto kern = mala_fwd_kernel<D, kScreen>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  if (e != cudaSuccess) return e;
+  kern<<<grid, C::THREADS, C::SMEM, stream>>>(tq, tk, tv, p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_fwd_bf16(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                            const FwdParams& p, int d, bool screen, int grid,
+                            cudaStream_t stream) {
+  if (d == 128)
+    return screen ? launch_fwd_impl<128, true>(tq, tk, tv, p, grid, stream)
+                  : launch_fwd_impl<128, false>(tq, tk, tv, p, grid, stream);
+  return screen ? launch_fwd_impl<64, true>(tq, tk, tv, p, grid, stream)
+                : launch_fwd_impl<64, false>(tq, tk, tv, p, grid, stream);
+}
+
+}  // namespace mala

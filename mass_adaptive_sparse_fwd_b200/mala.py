@@ -1,0 +1,183 @@
+"""Thin ctypes binding of the MALA C ABI (``include/mala.h``).
+
+Argument marshalling only: every step of forward, backward and decode runs in the
+CUDA kernels of ``libmala_b200.so``.  PyTorch supplies device memory and the current
+stream.  There is no fallback: if the library is missing the import of this module
+fails loudly.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+from . import build as _build
+
+_LIB_PATH = _build.LIB
+
+MALA_OK = 0
+STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported shape or dtype", 3: "CUDA error",
+          4: "device wait timed out", 5: "workspace too small"}
+MALA_BF16, MALA_FP32 = 0, 1
+MALA_FLAG_ALWAYS_TEST = 1
+TILE = 128
+
+EXPORTED = ("mala_fwd", "mala_bwd", "mala_decode", "mala_fwd_workspace_bytes",
+            "mala_bwd_workspace_bytes", "mala_decode_workspace_bytes", "mala_decode_num_splits",
+            "mala_read_device_error", "mala_set_wait_budget_ns", "mala_status_string",
+            "mala_version")
+
+
+class MalaError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn}: {STATUS.get(status, status)} (status {status})")
+        self.status = status
+
+
+def load_library(path: str = _LIB_PATH) -> ctypes.CDLL:
+    if not os.path.exists(path):
+        raise ImportError(f"MALA CUDA library not built: {path} (run python -m "
+                          "mass_adaptive_sparse_fwd_b200.build)")
+    lib = ctypes.CDLL(path)
+    vp, ci, cf, cu, sz = (ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_uint,
+                          ctypes.c_size_t)
+    lib.mala_fwd.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, cf, cf, cu, vp, sz, vp, vp]
+    lib.mala_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, cf, cf,
+                             cu, vp, sz, vp, vp]
+    lib.mala_decode.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, cf, cf, ci, cu, vp, sz,
+                                vp, vp]
+    for f in ("mala_fwd", "mala_bwd", "mala_decode", "mala_read_device_error",
+              "mala_set_wait_budget_ns"):
+        getattr(lib, f).restype = ci
+    lib.mala_fwd_workspace_bytes.argtypes = [ci] * 6
+    lib.mala_bwd_workspace_bytes.argtypes = [ci] * 6
+    lib.mala_decode_workspace_bytes.argtypes = [ci] * 7
+    for f in ("mala_fwd_workspace_bytes", "mala_bwd_workspace_bytes",
+              "mala_decode_workspace_bytes"):
+        getattr(lib, f).restype = sz
+    lib.mala_decode_num_splits.argtypes = [ci] * 4
+    lib.mala_decode_num_splits.restype = ci
+    lib.mala_read_device_error.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_uint32), ci]
+    lib.mala_set_wait_budget_ns.argtypes = [ctypes.c_uint64]
+    lib.mala_status_string.argtypes = [ci]
+    lib.mala_status_string.restype = ctypes.c_char_p
+    lib.mala_version.restype = ci
+    return lib
+
+
+_lib = load_library()
+
+
+def lib() -> ctypes.CDLL:
+    return _lib
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return MALA_BF16
+    if t.dtype == torch.float32:
+        return MALA_FP32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(fn: str, status: int):
+    if status != MALA_OK:
+        raise MalaError(fn, status)
+
+
+def n_tiles(n: int) -> int:
+    return (n + TILE - 1) // TILE
+
+
+def fwd_workspace_bytes(B, H, H_kv, L, d, dtype=MALA_BF16) -> int:
+    return _lib.mala_fwd_workspace_bytes(B, H, H_kv, L, d, dtype)
+
+
+def bwd_workspace_bytes(B, H, H_kv, L, d, dtype=MALA_BF16) -> int:
+    return _lib.mala_bwd_workspace_bytes(B, H, H_kv, L, d, dtype)
+
+
+def decode_workspace_bytes(B, H, H_kv, Nk, d, dtype=MALA_BF16, num_splits=0) -> int:
+    return _lib.mala_decode_workspace_bytes(B, H, H_kv, Nk, d, dtype, num_splits)
+
+
+def decode_num_splits(B, H, H_kv, Nk) -> int:
+    return _lib.mala_decode_num_splits(B, H, H_kv, Nk)
+
+
+def alloc_workspace(nbytes: int, device) -> torch.Tensor:
+    """A zeroed workspace buffer (uint8) suitable for any MALA call of that size."""
+    return torch.zeros(nbytes, dtype=torch.uint8, device=device)
+
+
+def mala_fwd(Q, K, V, scale, tau, O=None, LSE=None, flags=0, workspace=None, tile_mask=None,
+             stream=None):
+    """MALA forward through the C ABI.  Q [B,L,H,d], K/V [B,L,H_kv,d] (bf16 or fp32,
+    contiguous, on the GPU).  Returns (O, LSE)."""
+    B, L, H, d = Q.shape
+    H_kv = K.shape[2]
+    if O is None:
+        O = torch.empty_like(Q)
+    if LSE is None:
+        LSE = torch.empty((B, H, L), dtype=torch.float32, device=Q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel()
+    st = _lib.mala_fwd(_ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(LSE), B, H, H_kv, L, d,
+                       _dtype_code(Q), float(scale), float(tau), flags, _ptr(workspace), ws_bytes,
+                       _ptr(tile_mask), _stream(stream))
+    _check("mala_fwd", st)
+    return O, LSE
+
+
+def mala_bwd(Q, K, V, O, LSE, dO, scale, tau, dQ=None, dK=None, dV=None, flags=0,
+             workspace=None, tile_mask=None, stream=None):
+    """MALA backward through the C ABI.  Returns (dQ, dK, dV)."""
+    B, L, H, d = Q.shape
+    H_kv = K.shape[2]
+    dQ = torch.empty_like(Q) if dQ is None else dQ
+    dK = torch.empty_like(K) if dK is None else dK
+    dV = torch.empty_like(V) if dV is None else dV
+    ws_bytes = 0 if workspace is None else workspace.numel()
+    st = _lib.mala_bwd(_ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(LSE), _ptr(dO), _ptr(dQ), _ptr(dK),
+                       _ptr(dV), B, H, H_kv, L, d, _dtype_code(Q), float(scale), float(tau), flags,
+                       _ptr(workspace), ws_bytes, _ptr(tile_mask), _stream(stream))
+    _check("mala_bwd", st)
+    return dQ, dK, dV
+
+
+def mala_decode(q, Kc, Vc, scale, tau, num_splits=0, O=None, LSE=None, flags=0, workspace=None,
+                tile_mask=None, stream=None):
+    """MALA split-KV decode through the C ABI.  q [B,H,d]; Kc/Vc [B,N_k,H_kv,d].
+    Returns (O [B,H,d], LSE [B,H])."""
+    B, H, d = q.shape
+    Nk, H_kv = Kc.shape[1], Kc.shape[2]
+    O = torch.empty_like(q) if O is None else O
+    LSE = torch.empty((B, H), dtype=torch.float32, device=q.device) if LSE is None else LSE
+    ws_bytes = 0 if workspace is None else workspace.numel()
+    st = _lib.mala_decode(_ptr(q), _ptr(Kc), _ptr(Vc), _ptr(O), _ptr(LSE), B, H, H_kv, Nk, d,
+                          _dtype_code(q), float(scale), float(tau), int(num_splits), flags,
+                          _ptr(workspace), ws_bytes, _ptr(tile_mask), _stream(stream))
+    _check("mala_decode", st)
+    return O, LSE
+
+
+def read_device_error(workspace: torch.Tensor, clear: bool = True, stream=None) -> int:
+    out = ctypes.c_uint32(0)
+    _check("mala_read_device_error",
+           _lib.mala_read_device_error(_ptr(workspace), _stream(stream), ctypes.byref(out),
+                                       int(clear)))
+    return out.value
+
+
+def set_wait_budget_ns(ns: int):
+    _check("mala_set_wait_budget_ns", _lib.mala_set_wait_budget_ns(int(ns)))

@@ -1,0 +1,104 @@
+"""GPU parity of the MALA forward (C ABI -> sm_100a kernels) against the fp64 oracle."""
+
+import numpy as np
+import pytest
+import torch
+
+from mass_adaptive_sparse_fwd_b200 import synth
+from tests import parity as P
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def mala():
+    if not torch.cuda.is_available():
+        pytest.skip("no GPU")
+    from mass_adaptive_sparse_fwd_b200 import mala as m
+
+    return m
+
+
+def run_fwd(mala, inp, w, tau, flags=0):
+    Q, K, V = (P.to_dev(inp[k], w.dtype) for k in ("Q", "K", "V"))
+    B, L, H, d = Q.shape
+    T = mala.n_tiles(L)
+    mask = torch.full((B, H, T, T), 255, dtype=torch.uint8, device="cuda")
+    ws = mala.alloc_workspace(mala.fwd_workspace_bytes(B, H, K.shape[2], L, d), "cuda")
+    O, LSE = mala.mala_fwd(Q, K, V, w.scale, tau, flags=flags, workspace=ws, tile_mask=mask)
+    torch.cuda.synchronize()
+    assert mala.read_device_error(ws) == 0
+    return O.float().cpu().numpy(), LSE.cpu().numpy(), mask.cpu().numpy()
+
+
+def check_fwd(orc, mala, w, inp, tau, units=None, flags=0):
+    O, LSE, mask = run_fwd(mala, inp, w, tau, flags)
+    B, L, H, d = inp["Q"].shape
+    T = (L + 127) // 128
+    legal_all = P.fwd_legal(B, H, T)
+    # untouched entries only above the diagonal; decisions are 0/1 on legal tiles
+    assert (mask[~legal_all] == 255).all()
+    assert np.isin(mask[legal_all], (0, 1)).all()
+    force = np.where(legal_all, mask.astype(np.int16), -1).astype(np.int8)
+    oO, oLSE, omask, omargin = orc.mala_fwd(inp["Q"], inp["K"], inp["V"], w.scale, tau,
+                                            units=units, force=force)
+    legal = P.fwd_legal(B, H, T, units)
+    band = P.tile_bands(inp["Q"], inp["K"], w.scale, H // inp["K"].shape[2])
+    n, near, bad, worst = P.compare_masks(mask, omargin, band, legal)
+    assert bad == 0, f"{bad} tile decisions differ beyond the band (worst margin {worst})"
+    rows = np.isfinite(oLSE)  # [B,H,L] rows the oracle computed
+    rows_o = np.transpose(rows, (0, 2, 1))  # [B,L,H]
+    P.check_output(O, oO, rows_o)
+    assert np.abs(LSE - oLSE)[rows].max() < P.LSE_ABS
+    if tau == 0:
+        assert (mask[legal_all] == 1).all()
+    return {"tiles": n, "near": near, "retained": float(mask[legal_all].mean())}
+
+
+@pytest.mark.parametrize("tau", [0.0, 1.0])
+@pytest.mark.parametrize("shape", [
+    dict(B=1, H=4, Hkv=2, L=256, d=128, structure="peaked"),   # 2 tiles, GQA pairs
+    dict(B=2, H=6, Hkv=2, L=300, d=64, structure="normal"),    # ragged tail, odd group
+    dict(B=1, H=2, Hkv=2, L=384, d=128, structure="peaked"),   # G = 1: one slot idle
+])
+def test_fwd_small(orc, mala, shape, tau):
+    w, inp = synth.small_training(**shape)
+    check_fwd(orc, mala, w, inp, tau)
+
+
+def test_fwd_always_test_flag_at_tau0(orc, mala):
+    w, inp = synth.small_training(B=1, H=4, Hkv=1, L=512, d=128, structure="peaked")
+    st = check_fwd(orc, mala, w, inp, 0.0, flags=1)
+    assert st["retained"] == 1.0
+
+
+def test_fwd_peaked1k_full(orc, mala):
+    w = synth.WORKLOADS["peaked1k"]
+    inp = synth.make_training(w)
+    # at L = 1024 the 4 random prefix keys of 128 rows land in every earlier tile, so
+    # the oracle (and the kernel) retain all tiles here; decisions still must agree
+    check_fwd(orc, mala, w, inp, 1.0)
+
+
+def _units(B, H, T, n, seed):
+    rng = np.random.default_rng(seed)
+    u = {(B - 1, H - 1, T - 1), (0, 0, 0), (0, H // 2, T // 2)}
+    while len(u) < n:
+        u.add((int(rng.integers(B)), int(rng.integers(H)), int(rng.integers(T))))
+    return sorted(u)
+
+
+@pytest.mark.parametrize("tau", [1.0, 0.0, 1e-4, 1e-3])
+def test_fwd_mixed8k_sampled(orc, mala, tau):
+    w = synth.WORKLOADS["mixed8k"]
+    inp = synth.make_training(w)
+    T = w.L // 128
+    check_fwd(orc, mala, w, inp, tau, units=_units(w.B, w.H, T, 6, seed=int(tau * 1e4) + 1))
+
+
+@pytest.mark.slow
+def test_fwd_sinkband32k_sampled(orc, mala):
+    w = synth.WORKLOADS["sinkband32k"]
+    inp = synth.make_training(w)
+    T = w.L // 128
+    check_fwd(orc, mala, w, inp, 1.0, units=_units(w.B, w.H, T, 4, seed=5))
