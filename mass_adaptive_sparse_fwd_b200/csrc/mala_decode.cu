@@ -1,20 +1,560 @@
-// MALA split-KV decode (placeholder until the sm_100a kernel lands).
+// MALA split-KV decode kernel for sm_100a (bf16, head dim 64 or 128).
+//
+// "MassAlloc Attention: Let Attention Allocate Its Own Compute", §2.1 (L_0 = N_k in
+// decoding), §2.4 and A.1 (fused decoding: every cached key is scored, V is loaded and
+// P.V executed only for retained tiles; each split tests against its own partial
+// normaliser; the partial outputs are merged by the normaliser-aware reduction).
+//
+// Work unit = (batch b, KV head g, split s): the G = H / H_kv query heads of group g
+// against the split's key tiles, newest first.  Persistent CTAs walk the units
+// round-robin; the last CTA to finish a (b, g) merges its splits (atomic ticket).
+//
+// Decode is bound by HBM bandwidth: every K byte must be read, and V bytes only for
+// retained tiles.  The retention decisions depend on Q and K alone, so the kernel
+// decides ahead of the P.V work and gates each V load on the decision:
+//   warp 4      K producer: streams K tiles of the CTA's units into a ring (TMA).
+//   warp 5      V producer: waits for the decision of each tile and loads V only when
+//               at least one head of the group retains it.
+//   warps 0-3   consumers: scores S = K_t q_g^T (mma.sync m16n8k16, heads padded to
+//               8 as the N dimension), per-head tile maxima, retention test, online
+//               softmax state and P_t; the P.V product of tile t is done LAG tiles
+//               later, when its V has had time to arrive.
+// The contraction per tile is tiny (128 keys x 128 dims x G heads) and the kernel is
+// bandwidth bound, so it uses warp-level mma.sync rather than tcgen05 / TMEM.
+
+#include <cuda.h>
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
+
+#include <cmath>
+
 #include "mala.h"
 #include "mala_common.cuh"
+#include "sm100.cuh"
+
 namespace mala {
+
+bool make_tile_map(CUtensorMap* m, const void* base, int n0, int n1, int n2, int n3);
+int sm_count();
+
+namespace {
+
+constexpr int kDecThreads = 192;
+constexpr int kLag = 2;        // tiles between a decision and its P.V
+constexpr int kPR = kLag + 1;  // P / decision ring depth
+
+template <int D>
+struct DecCfg {
+  static constexpr int TILE_BYTES = kTile * D * 2;
+  static constexpr int BOXES = D / 64;
+  static constexpr int NK = (D == 128) ? 3 : 6;
+  static constexpr int NV = (D == 128) ? 3 : 6;
+  static constexpr int SMEM = (NK + NV) * TILE_BYTES + 1024;
+};
+
+struct DecParams {
+  int B, H, Hkv, Nk, T, G, S, n_units;
+  float scale_log2, thr2;  // thr2 = log2(tau / N_k), -inf when tau == 0
+  const __nv_bfloat16* q;  // [B, H, D]
+  __nv_bfloat16* O;        // [B, H, D]
+  float* LSE;              // [B, H]
+  float* part_o;           // [B, H, S, D]
+  float* part_z;           // [B, H, S] (natural log)
+  uint32_t* tickets;       // [B * Hkv]
+  uint8_t* tile_mask;      // [B, H, T] or null
+  uint32_t* err;
+  uint64_t budget_ns;
+};
+
+struct DecShared {
+  uint64_t k_full[6], k_empty[6], v_full[6], v_empty[6];
+  uint64_t dec_full[kPR], dec_empty[kPR];
+  __nv_bfloat16 qs[8][128];           // query rows of the group, heads >= G are zero
+  __nv_bfloat16 P[kPR][8][kTile];     // P_t, rows = heads (>= G zero)
+  float alpha[kPR][8];                // rescale of O at tile t, per head
+  uint32_t keep[kPR];                 // bit h: head h retained tile t
+  float red[4][8];                    // per-warp partial max / sum
+  uint32_t last_flag;
+  uint32_t abort_flag;
+};
+
+__device__ __forceinline__ void ldmatrix_x4(uint32_t addr, uint32_t& r0, uint32_t& r1,
+                                            uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
+__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t addr, uint32_t& r0, uint32_t& r1,
+                                                  uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
+__device__ __forceinline__ void mma_bf16(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                         uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Byte address of 16-byte chunk `c` (of 8 bf16 along the head dim) of key row `r` in
+// a tile loaded by TMA as D/64 boxes of [128 rows x 128 bytes] with 128-byte swizzle.
+__device__ __forceinline__ uint32_t tile_chunk_addr(uint32_t base, int r, int c) {
+  return base + (c >> 3) * 16384 + sw128_offset(r, c & 7);
+}
+
+__device__ __forceinline__ void unit_coords(const DecParams& p, int u, int& b, int& g, int& s,
+                                            int& t_lo, int& t_hi) {
+  s = u % p.S;
+  const int bg = u / p.S;
+  g = bg % p.Hkv;
+  b = bg / p.Hkv;
+  t_lo = static_cast<int>(static_cast<long long>(s) * p.T / p.S);
+  t_hi = static_cast<int>(static_cast<long long>(s + 1) * p.T / p.S);
+}
+
+template <int D, bool kScreen>
+__global__ void __launch_bounds__(kDecThreads, 1)
+    mala_decode_kernel(const __grid_constant__ CUtensorMap tmK,
+                       const __grid_constant__ CUtensorMap tmV, const DecParams p) {
+  using C = DecCfg<D>;
+  constexpr int NK = C::NK, NV = C::NV;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* sK = smem;
+  uint8_t* sV = smem + NK * C::TILE_BYTES;
+  __shared__ DecShared sh;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (tid == 0) {
+    for (int i = 0; i < NK; ++i) {
+      mbar_init(&sh.k_full[i], 1);
+      mbar_init(&sh.k_empty[i], 4);
+    }
+    for (int i = 0; i < NV; ++i) {
+      mbar_init(&sh.v_full[i], 1);
+      mbar_init(&sh.v_empty[i], 4);
+    }
+    for (int i = 0; i < kPR; ++i) {
+      mbar_init(&sh.dec_full[i], 1);
+      mbar_init(&sh.dec_empty[i], 1);
+    }
+    sh.abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  const AbortState ast{&sh.abort_flag, p.err, p.budget_ns, 0x300u};
+
+  if (warp == 4) {
+    // ------------------------------------------------------------------ K producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tmK);
+      uint32_t c = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+        int b, g, s, t_lo, t_hi;
+        unit_coords(p, u, b, g, s, t_lo, t_hi);
+        for (int t = t_hi - 1; t >= t_lo && ok; --t, ++c) {
+          const int st = c % NK;
+          if (c >= NK && !(ok = mbar_wait(&sh.k_empty[st], ((c / NK) - 1) & 1, ast, 1))) break;
+          mbar_arrive_expect_tx(&sh.k_full[st], C::TILE_BYTES);
+          for (int x = 0; x < C::BOXES; ++x)
+            tma_load_4d(sK + st * C::TILE_BYTES + x * 16384, &tmK, &sh.k_full[st], x * 64, g,
+                        t * kTile, b);
+        }
+      }
+      if (!ok) {
+        AbortState drain = ast;
+        uint32_t zero = 0;
+        drain.flag = &zero;
+        drain.budget_ns = 200000000ull;
+        for (uint32_t cc = (c > NK ? c - NK : 0); cc < c; ++cc)
+          mbar_wait(&sh.k_full[cc % NK], (cc / NK) & 1, drain, 2);
+      }
+    }
+  } else if (warp == 5) {
+    // ------------------------------------------------------------------ V producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tmV);
+      uint32_t n = 0, c = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+        int b, g, s, t_lo, t_hi;
+        unit_coords(p, u, b, g, s, t_lo, t_hi);
+        for (int t = t_hi - 1; t >= t_lo && ok; --t, ++n) {
+          const int slot = n % kPR;
+          if (!(ok = mbar_wait(&sh.dec_full[slot], (n / kPR) & 1, ast, 3))) break;
+          const uint32_t keep = sh.keep[slot];
+          mbar_arrive(&sh.dec_empty[slot]);
+          if (!keep) continue;
+          const int st = c % NV;
+          if (c >= NV && !(ok = mbar_wait(&sh.v_empty[st], ((c / NV) - 1) & 1, ast, 4))) break;
+          mbar_arrive_expect_tx(&sh.v_full[st], C::TILE_BYTES);
+          for (int x = 0; x < C::BOXES; ++x)
+            tma_load_4d(sV + st * C::TILE_BYTES + x * 16384, &tmV, &sh.v_full[st], x * 64, g,
+                        t * kTile, b);
+          ++c;
+        }
+      }
+      if (!ok) {
+        AbortState drain = ast;
+        uint32_t zero = 0;
+        drain.flag = &zero;
+        drain.budget_ns = 200000000ull;
+        for (uint32_t cc = (c > NV ? c - NV : 0); cc < c; ++cc)
+          mbar_wait(&sh.v_full[cc % NV], (cc / NV) & 1, drain, 5);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------------ consumers
+    const int G = p.G;
+    const float NEG_INF = -INFINITY;
+    const uint32_t sKa = smem_u32(sK), sVa = smem_u32(sV);
+    uint32_t kc = 0, vc = 0, n_glob = 0;
+    bool ok = true;
+    // zero the padded heads of P once (rows >= G are never written again)
+    for (int i = tid; i < kPR * 8 * kTile; i += 128) {
+      const int row = (i / kTile) % 8;
+      if (row >= G) (&sh.P[0][0][0])[i] = __float2bfloat16(0.f);
+    }
+    for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+      int b, g, s, t_lo, t_hi;
+      unit_coords(p, u, b, g, s, t_lo, t_hi);
+      const int nt = t_hi - t_lo;
+      // query rows of the group -> shared, then the B fragments of S = K q^T
+      named_bar_sync(1, 128);
+      for (int i = tid; i < 8 * D; i += 128) {
+        const int hh = i / D, c = i % D;
+        sh.qs[hh][c] = (hh < G) ? p.q[(static_cast<size_t>(b) * p.H + g * G + hh) * D + c]
+                                : __float2bfloat16(0.f);
+      }
+      named_bar_sync(1, 128);
+      uint32_t qb[D / 16][2];
+#pragma unroll
+      for (int ks = 0; ks < D / 16; ++ks) {
+        const int hh = lane >> 2, c0 = ks * 16 + (lane & 3) * 2;
+        qb[ks][0] = *reinterpret_cast<const uint32_t*>(&sh.qs[hh][c0]);
+        qb[ks][1] = *reinterpret_cast<const uint32_t*>(&sh.qs[hh][c0 + 8]);
+      }
+      // per-head running state (replicated in every consumer thread)
+      float m[4], l[4];
+#pragma unroll
+      for (int hh = 0; hh < 4; ++hh) { m[hh] = NEG_INF; l[hh] = 0.f; }
+      // O^T accumulators: warp owns head-dim rows [w*D/4, (w+1)*D/4)
+      constexpr int MB = D / 64;  // 16-row blocks per warp
+      float acc[MB][4];
+#pragma unroll
+      for (int mb = 0; mb < MB; ++mb)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[mb][e] = 0.f;
+
+      for (int n = 0; n < nt + kLag && ok; ++n) {
+        if (n < nt) {
+          const int t = t_hi - 1 - n;
+          const uint32_t slot = (n_glob + n) % kPR;
+          const int kst = kc % NK;
+          // A failed wait only raises the abort flag; the consumers leave the loop
+          // together, right after their next named barrier.
+          const bool got = __all_sync(0xffffffffu, mbar_wait(&sh.k_full[kst], (kc / NK) & 1, ast, 10));
+          // scores of this warp's 32 keys x 8 (padded) heads
+          float sc[2][4];
+#pragma unroll
+          for (int kb = 0; kb < 2; ++kb) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) sc[kb][e] = 0.f;
+            const int row0 = warp * 32 + kb * 16;
+            if (got) {
+#pragma unroll
+              for (int ks = 0; ks < D / 16; ++ks) {
+                uint32_t a0, a1, a2, a3;
+                ldmatrix_x4(tile_chunk_addr(sKa + kst * C::TILE_BYTES, row0 + (lane & 15),
+                                            ks * 2 + (lane >> 4)),
+                            a0, a1, a2, a3);
+                mma_bf16(sc[kb], a0, a1, a2, a3, qb[ks][0], qb[ks][1]);
+              }
+            }
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sh.k_empty[kst]);
+          ++kc;
+          // scale into log2 units, mask keys past the end, per-head tile maxima
+          float mx[2] = {NEG_INF, NEG_INF};
+#pragma unroll
+          for (int kb = 0; kb < 2; ++kb)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int key = t * kTile + warp * 32 + kb * 16 + (lane >> 2) + (e >> 1) * 8;
+              float x = sc[kb][e] * p.scale_log2;
+              x = (key < p.Nk) ? x : NEG_INF;
+              sc[kb][e] = x;
+              mx[e & 1] = fmaxf(mx[e & 1], x);
+            }
+#pragma unroll
+          for (int o = 4; o < 32; o <<= 1) {
+            mx[0] = fmaxf(mx[0], __shfl_xor_sync(0xffffffffu, mx[0], o));
+            mx[1] = fmaxf(mx[1], __shfl_xor_sync(0xffffffffu, mx[1], o));
+          }
+          if (lane < 2) {  // lanes 0, 1 hold heads 0-1 and 2-3
+            sh.red[warp][lane * 2] = mx[0];
+            sh.red[warp][lane * 2 + 1] = mx[1];
+          }
+          named_bar_sync(1, 128);
+          if (*ast.flag) { ok = false; break; }
+          // retention test per head (Eq. 3 with L_0 = N_k), identical in every thread
+          uint32_t keep = 0;
+          float mnew[4], alpha[4];
+#pragma unroll
+          for (int hh = 0; hh < 4; ++hh) {
+            const float tmax = fmaxf(fmaxf(sh.red[0][hh], sh.red[1][hh]),
+                                     fmaxf(sh.red[2][hh], sh.red[3][hh]));
+            bool k = hh < G;
+            if (kScreen && k) k = (l[hh] == 0.f) || (tmax >= m[hh] + __log2f(l[hh]) + p.thr2);
+            mnew[hh] = m[hh];
+            alpha[hh] = 1.f;
+            if (k) {
+              keep |= 1u << hh;
+              if (tmax > m[hh] + 8.0f) {
+                mnew[hh] = tmax;
+                alpha[hh] = fast_exp2(m[hh] - tmax);  // 0 on the first retained tile
+              }
+            }
+          }
+          // hand the decision to the V producer (ring slot must be free)
+          if (tid == 0) {
+            bool free_slot = true;
+            if (n_glob + n >= kPR)
+              free_slot = mbar_wait(&sh.dec_empty[slot], (((n_glob + n) / kPR) - 1) & 1, ast, 11);
+            sh.keep[slot] = keep;
+            if (free_slot) mbar_arrive(&sh.dec_full[slot]);
+          }
+          if (p.tile_mask && tid < G)
+            p.tile_mask[(static_cast<size_t>(b) * p.H + g * G + tid) * p.T + t] =
+                (keep >> tid) & 1u;
+          if (keep) {
+            // P_t for retained heads (zero for the others) and its row sums
+            float ps[2] = {0.f, 0.f};
+            const int h0 = (lane & 3) * 2;
+#pragma unroll
+            for (int kb = 0; kb < 2; ++kb)
+#pragma unroll
+              for (int r8 = 0; r8 < 2; ++r8) {
+                const int key = warp * 32 + kb * 16 + (lane >> 2) + r8 * 8;
+#pragma unroll
+                for (int c = 0; c < 2; ++c) {
+                  const int hh = h0 + c;
+                  float pv = 0.f;
+                  if (hh < 4 && ((keep >> hh) & 1u)) {
+                    const float mu = (mnew[hh] == NEG_INF) ? 0.f : mnew[hh];
+                    pv = fast_exp2(sc[kb][r8 * 2 + c] - mu);
+                  }
+                  ps[c] += pv;
+                  if (hh < G) sh.P[slot][hh][key] = __float2bfloat16(pv);
+                }
+              }
+#pragma unroll
+            for (int o = 4; o < 32; o <<= 1) {
+              ps[0] += __shfl_xor_sync(0xffffffffu, ps[0], o);
+              ps[1] += __shfl_xor_sync(0xffffffffu, ps[1], o);
+            }
+            named_bar_sync(1, 128);  // everyone has read sh.red (maxima)
+            if (lane < 2) {
+              sh.red[warp][lane * 2] = ps[0];
+              sh.red[warp][lane * 2 + 1] = ps[1];
+            }
+            if (tid < 8) sh.alpha[slot][tid] = (tid < 4) ? alpha[tid] : 1.f;
+            named_bar_sync(1, 128);
+#pragma unroll
+            for (int hh = 0; hh < 4; ++hh) {
+              if ((keep >> hh) & 1u) {
+                const float tsum = sh.red[0][hh] + sh.red[1][hh] + sh.red[2][hh] + sh.red[3][hh];
+                l[hh] = l[hh] * alpha[hh] + tsum;
+                m[hh] = mnew[hh];
+              }
+            }
+          }
+          named_bar_sync(1, 128);  // sh.red is reused by the next tile
+          if (*ast.flag) { ok = false; break; }
+        }
+        // P.V of the tile decided kLag iterations ago
+        if (n >= kLag) {
+          const int n2 = n - kLag;
+          const uint32_t slot2 = (n_glob + n2) % kPR;
+          const uint32_t keep2 = sh.keep[slot2];
+          if (keep2) {
+            const int vst = vc % NV;
+            const bool vgot =
+                __all_sync(0xffffffffu, mbar_wait(&sh.v_full[vst], (vc / NV) & 1, ast, 12));
+            // rescale: thread's accumulator columns are heads (lane&3)*2 + {0,1}
+            const int h0 = (lane & 3) * 2;
+            const float a0 = (h0 < 4) ? sh.alpha[slot2][h0] : 1.f;
+            const float a1 = (h0 + 1 < 4) ? sh.alpha[slot2][h0 + 1] : 1.f;
+#pragma unroll
+            for (int mb = 0; mb < MB; ++mb) {
+              acc[mb][0] *= a0; acc[mb][1] *= a1; acc[mb][2] *= a0; acc[mb][3] *= a1;
+            }
+            const uint32_t vbase = sVa + vst * C::TILE_BYTES;
+#pragma unroll
+            for (int ks = 0; ks < (vgot ? kTile / 16 : 0); ++ks) {
+              const int hh = lane >> 2, kk = ks * 16 + (lane & 3) * 2;
+              const uint32_t b0 = *reinterpret_cast<const uint32_t*>(&sh.P[slot2][hh][kk]);
+              const uint32_t b1 = *reinterpret_cast<const uint32_t*>(&sh.P[slot2][hh][kk + 8]);
+#pragma unroll
+              for (int mb = 0; mb < MB; ++mb) {
+                const int d0 = warp * (D / 4) + mb * 16;
+                const int mi = lane >> 3;
+                uint32_t r0, r1, r2, r3;
+                ldmatrix_x4_trans(
+                    tile_chunk_addr(vbase, ks * 16 + (lane & 7) + (mi >> 1) * 8, (d0 >> 3) + (mi & 1)),
+                    r0, r1, r2, r3);
+                mma_bf16(acc[mb], r0, r1, r2, r3, b0, b1);
+              }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sh.v_empty[vst]);
+            ++vc;
+          } else {
+            // nothing retained: O keeps its scale (alpha = 1 for every head)
+          }
+        }
+      }
+      if (!ok) break;
+      n_glob += nt;
+      named_bar_sync(1, 128);
+      if (*ast.flag) { ok = false; break; }
+      // this split's normalised output o_s = acc / l and z_s = (m + log2 l) ln 2
+      {
+        const int h0 = (lane & 3) * 2;
+#pragma unroll
+        for (int mb = 0; mb < MB; ++mb)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int hh = h0 + (e & 1);
+            const int dd = warp * (D / 4) + mb * 16 + (lane >> 2) + (e >> 1) * 8;
+            if (hh < G) {
+              const float lv = (hh == 0) ? l[0] : (hh == 1) ? l[1] : (hh == 2) ? l[2] : l[3];
+              p.part_o[((static_cast<size_t>(b) * p.H + g * G + hh) * p.S + s) * D + dd] =
+                  acc[mb][e] / lv;
+            }
+          }
+        if (tid < G)
+          p.part_z[(static_cast<size_t>(b) * p.H + g * G + tid) * p.S + s] =
+              (m[tid] + __log2f(l[tid])) * kLn2;
+      }
+      // last CTA of this (b, g) merges the splits
+      named_bar_sync(1, 128);
+      if (tid == 0) {
+        __threadfence();
+        const uint32_t prev = atomicAdd(&p.tickets[b * p.Hkv + g], 1u);
+        sh.last_flag = (prev == static_cast<uint32_t>(p.S - 1)) ? 1u : 0u;
+      }
+      named_bar_sync(1, 128);
+      if (sh.last_flag) {
+        __threadfence();
+        for (int i = tid; i < G * D; i += 128) {
+          const int hh = i / D, dd = i % D;
+          const size_t row = static_cast<size_t>(b) * p.H + g * G + hh;
+          const volatile float* pz = p.part_z + row * p.S;
+          const volatile float* po = p.part_o + row * p.S * D;
+          float zmax = NEG_INF;
+          for (int ss = 0; ss < p.S; ++ss) zmax = fmaxf(zmax, pz[ss]);
+          float wsum = 0.f, o = 0.f;
+          for (int ss = 0; ss < p.S; ++ss) {
+            const float wgt = __expf(pz[ss] - zmax);
+            wsum += wgt;
+            o += wgt * po[ss * D + dd];
+          }
+          p.O[row * D + dd] = __float2bfloat16(o / wsum);
+          if (dd == 0) p.LSE[row] = zmax + __logf(wsum);
+        }
+      }
+    }
+  }
+  __syncthreads();
+}
+
+}  // namespace
+
 int decode_auto_splits(int B, int Hkv, int Nk) {
+  // about eight persistent-CTA waves on a 148-SM B200, at least 8 key tiles per split
   const int T = (Nk + kTile - 1) / kTile;
-  int s = (2 * 148 + B * Hkv - 1) / (B * Hkv);
-  return s < 1 ? 1 : (s > T ? T : s);
+  const int bg = B * Hkv;
+  int s = (8 * 148 + bg / 2) / bg;
+  const int cap = T / 8 > 1 ? T / 8 : 1;
+  if (s > cap) s = cap;
+  if (s < 1) s = 1;
+  if (s > T) s = T;
+  return s;
 }
+
 size_t decode_workspace_bytes(int B, int H, int Hkv, int Nk, int d, int dtype, int S) {
-  (void)Hkv; (void)Nk; (void)dtype;
-  return kWorkspaceHeader + (size_t)B * H * S * (d + 1) * 4;
+  (void)Nk; (void)dtype;
+  const size_t part = static_cast<size_t>(B) * H * S * (d + 1) * sizeof(float);
+  const size_t tick = static_cast<size_t>(B) * Hkv * sizeof(uint32_t);
+  return kWorkspaceHeader + ((part + 255) / 256) * 256 + ((tick + 255) / 256) * 256;
 }
-mala_status decode_dispatch(const void*, const void*, const void*, void*, float*, int, int, int,
-                            int, int, int, float, float, int, unsigned, uint8_t*, uint8_t*,
-                            uint64_t, cudaStream_t) {
-  return MALA_ERR_UNSUPPORTED;
+
+mala_status fp32_decode(const float* q, const float* K, const float* V, float* O, float* LSE,
+                        int B, int H, int Hkv, int Nk, int d, float scale, float tau, int S,
+                        bool screen, uint8_t* ws, uint8_t* tile_mask, cudaStream_t stream);
+
+template <int D, bool kScreen>
+static cudaError_t launch_decode(const CUtensorMap& tk, const CUtensorMap& tv,
+                                 const DecParams& p, int grid, cudaStream_t stream) {
+  auto kern = mala_decode_kernel<D, kScreen>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       DecCfg<D>::SMEM);
+  if (e != cudaSuccess) return e;
+  kern<<<grid, kDecThreads, DecCfg<D>::SMEM, stream>>>(tk, tv, p);
+  return cudaGetLastError();
 }
+
+mala_status decode_dispatch(const void* q, const void* K, const void* V, void* O, float* LSE,
+                            int B, int H, int Hkv, int Nk, int d, int dtype, float scale,
+                            float tau, int num_splits, unsigned flags, uint8_t* ws,
+                            uint8_t* tile_mask, uint64_t budget_ns, cudaStream_t stream) {
+  const bool screen = (tau > 0.f) || (flags & MALA_FLAG_ALWAYS_TEST);
+  if (dtype == MALA_FP32)
+    return fp32_decode(static_cast<const float*>(q), static_cast<const float*>(K),
+                       static_cast<const float*>(V), static_cast<float*>(O), LSE, B, H, Hkv, Nk,
+                       d, scale, tau, num_splits, screen, ws, tile_mask, stream);
+  if (H / Hkv > 4) return MALA_ERR_UNSUPPORTED;  // the kernel packs up to 4 heads per group
+  CUtensorMap tk, tv;
+  if (!make_tile_map(&tk, K, d, Hkv, Nk, B) || !make_tile_map(&tv, V, d, Hkv, Nk, B))
+    return MALA_ERR_CUDA;
+  DecParams p;
+  p.B = B; p.H = H; p.Hkv = Hkv; p.Nk = Nk; p.T = (Nk + kTile - 1) / kTile; p.G = H / Hkv;
+  p.S = num_splits;
+  p.n_units = B * Hkv * num_splits;
+  p.scale_log2 = scale * kLog2e;
+  p.thr2 = (tau > 0.f) ? std::log2(tau) - std::log2(static_cast<float>(Nk)) : -INFINITY;
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.O = static_cast<__nv_bfloat16*>(O);
+  p.LSE = LSE;
+  uint8_t* part = ws + kWorkspaceHeader;
+  const size_t part_bytes = static_cast<size_t>(B) * H * num_splits * (d + 1) * sizeof(float);
+  p.part_o = reinterpret_cast<float*>(part);
+  p.part_z = p.part_o + static_cast<size_t>(B) * H * num_splits * d;
+  p.tickets = reinterpret_cast<uint32_t*>(part + ((part_bytes + 255) / 256) * 256);
+  p.tile_mask = tile_mask;
+  p.err = reinterpret_cast<uint32_t*>(ws) + kHdrError;
+  p.budget_ns = budget_ns;
+  if (cudaMemsetAsync(p.tickets, 0, static_cast<size_t>(B) * Hkv * sizeof(uint32_t), stream) !=
+      cudaSuccess)
+    return MALA_ERR_CUDA;
+  const int grid = p.n_units < sm_count() ? p.n_units : sm_count();
+  cudaError_t e;
+  if (d == 128)
+    e = screen ? launch_decode<128, true>(tk, tv, p, grid, stream)
+               : launch_decode<128, false>(tk, tv, p, grid, stream);
+  else
+    e = screen ? launch_decode<64, true>(tk, tv, p, grid, stream)
+               : launch_decode<64, false>(tk, tv, p, grid, stream);
+  return e == cudaSuccess ? MALA_OK : MALA_ERR_CUDA;
+}
+
 }  // namespace mala

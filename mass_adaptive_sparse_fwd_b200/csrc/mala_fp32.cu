@@ -7,3 +7,9 @@ mala_status fp32_fwd(const float*, const float*, const float*, float*, float*, i
   return MALA_ERR_UNSUPPORTED;
 }
 }  // namespace mala
+namespace mala {
+mala_status fp32_decode(const float*, const float*, const float*, float*, float*, int, int, int,
+                        int, int, float, float, int, bool, uint8_t*, uint8_t*, cudaStream_t) {
+  return MALA_ERR_UNSUPPORTED;
+}
+}  // namespace mala

@@ -292,7 +292,10 @@ __global__ void __launch_bounds__(384, 1)
     bool ok = true;
     for (uint32_t k = 0; ok; ++k) {
       const int ring = k & 1;
-      if (!(ok = mbar_wait(&sh.sched_full[ring], (k >> 1) & 1, ast, 20))) break;
+      // every exit of this loop is decided right after a warpgroup barrier, so that the
+      // 128 threads of the slot always leave together
+      const bool got = mbar_wait(&sh.sched_full[ring], (k >> 1) & 1, ast, 20);
+      if (named_bar_or(1 + s, 128, !got) || *ast.flag) { ok = false; break; }
       const int u = sh.sched_ring[ring];
       mbar_arrive(&sh.sched_empty[ring]);
       if (u >= p.n_units) break;
@@ -307,13 +310,22 @@ __global__ void __launch_bounds__(384, 1)
       const int n = w.i + 1;
       for (int t = 0; t < n; ++t) {
         const int j = w.i - t;
-        if (!(ok = mbar_wait(&sh.s_full[s], ns & 1, ast, 21))) break;
+        // A failed wait never leaves the loop before the next named barrier of the
+        // warpgroup: the abort flag is set and checked right after the vote.
+        const bool got = mbar_wait(&sh.s_full[s], ns & 1, ast, 21);
         ++ns;
         tc_fence_after();
         uint32_t v[4][32];
+        if (__all_sync(0xffffffffu, got)) {
 #pragma unroll
-        for (int cc = 0; cc < 4; ++cc) tmem_ld32(tS + cc * 32, v[cc]);
-        tmem_wait_ld();
+          for (int cc = 0; cc < 4; ++cc) tmem_ld32(tS + cc * 32, v[cc]);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int cc = 0; cc < 4; ++cc)
+#pragma unroll
+            for (int e = 0; e < 32; ++e) v[cc][e] = 0xff800000u;  // -inf
+        }
         float rmax = NEG_INF;
         if (t == 0 || !valid) {
           const int lim = valid ? r : -1;  // diagonal tile: keys c <= r are legal
@@ -340,6 +352,7 @@ __global__ void __launch_bounds__(384, 1)
         if (kScreen) {
           const bool mine = (rmax != NEG_INF) && (l == 0.f || rmax >= m2 + __log2f(l) + thr2);
           keep = named_bar_or(1 + s, 128, mine);
+          if (*ast.flag) { ok = false; break; }
         }
         if (p.tile_mask && r == 0)
           p.tile_mask[((static_cast<size_t>(w.b) * p.H + h) * p.T + w.i) * p.T + j] = keep ? 1 : 0;
@@ -358,9 +371,9 @@ __global__ void __launch_bounds__(384, 1)
         }
         const float m_use = (m_new == NEG_INF) ? 0.f : m_new;
         const float alpha = rescale ? fast_exp2(m2 - m_new) : 1.f;
-        if (__any_sync(0xffffffffu, rescale)) {
-          // the previous PV of this slot must have landed before O is touched
-          if (!(ok = mbar_wait(&sh.o_done[s], (npv - 1) & 1, ast, 22))) break;
+        if (__any_sync(0xffffffffu, rescale) &&
+            // the previous PV of this slot must have landed before O is touched
+            __all_sync(0xffffffffu, mbar_wait(&sh.o_done[s], (npv - 1) & 1, ast, 22))) {
           tc_fence_after();
 #pragma unroll
           for (int cc = 0; cc < D / 32; ++cc) {
@@ -395,9 +408,9 @@ __global__ void __launch_bounds__(384, 1)
       }
       if (!ok) break;
       // epilogue: O = acc / l, LSE = (m + log2 l) * ln 2
-      if (npv > npv_unit0) {
-        if (!(ok = mbar_wait(&sh.o_done[s], (npv - 1) & 1, ast, 23))) break;
-      }
+      bool o_ready = true;
+      if (npv > npv_unit0) o_ready = mbar_wait(&sh.o_done[s], (npv - 1) & 1, ast, 23);
+      if (!__all_sync(0xffffffffu, o_ready)) continue;  // aborting: the next vote exits
       tc_fence_after();
       const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
       __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.O) +

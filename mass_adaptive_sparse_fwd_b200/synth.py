@@ -30,7 +30,9 @@ V ~ N(0, 1) everywhere; dO is a Rademacher (+-1) probe.
 
 from __future__ import annotations
 
+import concurrent.futures as cf
 import math
+import os
 from dataclasses import dataclass, field
 
 import numpy as np
@@ -85,20 +87,46 @@ def _round(x: np.ndarray, dtype: str) -> np.ndarray:
     return round_bf16(x) if dtype == "bf16" else x
 
 
-def normal(seed: int, tensor: int, shape, dtype: str, chunk_axis0: bool = True) -> np.ndarray:
-    """N(0, 1) draws of ``shape``, generated in chunks along axis 0 (one key per chunk)."""
+_CHUNK = 1 << 22  # elements per generator chunk (each chunk has its own Philox key)
+
+
+def _chunked(shape, fill):
+    """Fills a float32 array of ``shape`` chunk by chunk (rows of the flattened leading
+    dimensions), in parallel threads; chunk c is always drawn from key c, so the result
+    does not depend on the thread count."""
+    shape = tuple(int(x) for x in shape)
     out = np.empty(shape, dtype=np.float32)
-    if chunk_axis0 and len(shape) > 1:
-        for c in range(shape[0]):
-            out[c] = _rng(seed, tensor, c).standard_normal(shape[1:], dtype=np.float32)
+    flat = out.reshape(-1, shape[-1]) if len(shape) > 1 else out.reshape(1, -1)
+    rows = flat.shape[0]
+    rows_per = max(1, _CHUNK // max(1, flat.shape[1]))
+    starts = list(range(0, rows, rows_per))
+
+    def work(c):
+        r0 = starts[c]
+        r1 = min(rows, r0 + rows_per)
+        flat[r0:r1] = fill(c, (r1 - r0, flat.shape[1]))
+
+    if len(starts) == 1:
+        work(0)
     else:
-        out[...] = _rng(seed, tensor).standard_normal(shape, dtype=np.float32)
-    return _round(out, dtype)
+        with cf.ThreadPoolExecutor(max_workers=min(16, os.cpu_count() or 1)) as ex:
+            list(ex.map(work, range(len(starts))))
+    return out
+
+
+def normal(seed: int, tensor: int, shape, dtype: str) -> np.ndarray:
+    """N(0, 1) draws of ``shape``, rounded to ``dtype``."""
+    def fill(c, sh):
+        x = _rng(seed, tensor, c).standard_normal(sh, dtype=np.float32)
+        return round_bf16(x) if dtype == "bf16" else x
+    return _chunked(shape, fill)
 
 
 def rademacher(seed: int, tensor: int, shape) -> np.ndarray:
-    bits = _rng(seed, tensor).integers(0, 2, size=shape, dtype=np.int8)
-    return (bits.astype(np.float32) * 2.0 - 1.0)
+    def fill(c, sh):
+        bits = _rng(seed, tensor, c).integers(0, 2, size=sh, dtype=np.int8)
+        return bits.astype(np.float32) * 2.0 - 1.0
+    return _chunked(shape, fill)
 
 
 def _peaked_queries(K: np.ndarray, heads, H: int, seed: int, dtype: str,
