@@ -1,15 +1,691 @@
-// MALA backward (placeholder until the sm_100a kernel lands).
+// MALA backward for sm_100a (bf16, head dim 64 or 128).
+//
+// "MassAlloc Attention: Let Attention Allocate Its Own Compute", §2.2 (offline sparse
+// probability, Eq. (4)), App. A Algorithm 2 and A.1 (fused backward execution).
+//
+// Three launches:
+//   1. mala_bwd_prep:  D_q = rowsum(O_q * dO_q) (fp32) and zeroing of the fp32 dQ
+//                      accumulator (the softmax-backward term of Algorithm 2).
+//   2. mala_bwd_kernel (below): key-major, one persistent CTA per SM pulling units
+//                      (b, KV head g, key block j) heaviest first (small j); within a
+//                      unit the G query heads of the group and the query blocks
+//                      i = j, j+1, ... are visited in ascending order (A.1).
+//   3. mala_bwd_dq:    dQ = bf16(dQ accumulator).
+//
+// Per tile (key block j, query block i of head h) the score tile S^T = K_j Q_i^T is
+// always recomputed.  The offline test of Eq. (4): the tile is retained iff some legal
+// entry has s_kq * scale - LSE_q >= log(tau / L_q) (L_q = q + 1), evaluated in log2
+// units.  Only a retained tile runs the post-score work:
+//   P^T = exp(S^T - LSE),  dP^T = V_j dO_i^T,  dS^T = P^T o (dP^T - D) * scale,
+//   dV += P^T dO_i,  dK += dS^T Q_i,  dQ_i += dS K_j  (fp32 reduction into global).
+//
+// Warp roles (512 threads):
+//   warp 0       TMA producer: K_j and V_j once per unit; Q_i and dO_i per tile
+//                (dO is fetched with Q, ahead of the decision, like V in the forward).
+//   warp 1       TMEM owner and UMMA issuer.
+//   warps 4-11   two softmax warpgroups: thread = key row (TMEM lane); warpgroup w
+//                owns query columns [64 w, 64 w + 64).  They evaluate the test (one
+//                bar.red.or over both groups), write P^T into TMEM and dS^T into shared
+//                memory.
+//   warps 12-15  dQ drain (TMEM -> red.global.add.v4.f32) and the per-unit dK / dV
+//                epilogue.
+// TMEM columns: S^T [0,128) (P^T bf16 overwrites [0,64)), dP^T [128,256) (the dQ tile
+// of the same step overwrites it once dS^T has been formed), dV [256, 256+D),
+// dK [256+D, 256+2D).
+
+#include <cuda.h>
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
+
+#include <cmath>
+
 #include "mala.h"
 #include "mala_common.cuh"
+#include "sm100.cuh"
+
 namespace mala {
+
+bool make_tile_map(CUtensorMap* m, const void* base, int n0, int n1, int n2, int n3);
+int sm_count();
+
+namespace {
+
+constexpr int kBwdThreads = 512;
+
+template <int D>
+struct BwdCfg {
+  static constexpr int TILE_BYTES = kTile * D * 2;
+  static constexpr int BOXES = D / 64;
+  static constexpr int NQ = 2;  // Q / dO ring stages
+  // K, V, NQ x (Q, dO), dS^T (128 x 128 bf16)
+  static constexpr int SMEM = 2 * TILE_BYTES + 2 * NQ * TILE_BYTES + kTile * kTile * 2;
+};
+
+struct BwdParams {
+  int B, H, Hkv, L, T, G, n_units;
+  float scale, scale_log2, log2_tau;
+  const float* LSE;      // [B, H, L] natural log
+  const float* Dsum;     // [B, H, L]
+  float* dQacc;          // [B, L, H, D] fp32
+  __nv_bfloat16* dK;     // [B, L, Hkv, D]
+  __nv_bfloat16* dV;
+  uint8_t* tile_mask;    // [B, H, T, T] or null
+  uint32_t* err;
+  uint32_t* sched;
+  uint64_t budget_ns;
+};
+
+struct BwdShared {
+  uint64_t kv_full, kv_empty;
+  uint64_t q_full[2], q_empty[2];
+  uint64_t s_full, p_full, dp_full, ds_full, dq_full, dq_empty, acc_full, acc_empty;
+  uint64_t sched_full[2], sched_empty[2];
+  uint64_t final_bar;
+  float c2[2][64];   // per softmax warpgroup: LSE2_q + log2(tau / L_q) (+inf if q >= L)
+  float lse2[2][64]; // LSE_q * log2(e)
+  float dsum[2][64]; // D_q
+  int sched_ring[2];
+  uint32_t dec;      // decision of the current tile (1 = retained)
+  uint32_t dq_flag[2];
+  uint32_t acc_valid;  // the unit retained at least one tile (dK / dV were written)
+  uint32_t tmem_base;
+  uint32_t abort_flag;
+};
+
+struct BUnit {
+  int b, g, j, ntiles;  // tiles = G heads x (T - j) query blocks
+};
+
+__device__ __forceinline__ BUnit decode_bunit(const BwdParams& p, int u) {
+  BUnit w;
+  const int nbg = p.B * p.Hkv;
+  w.j = u / nbg;
+  const int r = u % nbg;
+  w.b = r / p.Hkv;
+  w.g = r % p.Hkv;
+  w.ntiles = p.G * (p.T - w.j);
+  return w;
+}
+
+// tile n of a unit -> (head h, query block i)
+__device__ __forceinline__ void tile_hi(const BwdParams& p, const BUnit& w, int n, int& h,
+                                        int& i) {
+  const int per = p.T - w.j;
+  h = w.g * p.G + n / per;
+  i = w.j + n % per;
+}
+
+__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b),
+               "f"(c), "f"(d)
+               : "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+template <int D, bool kScreen>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    mala_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
+                    const BwdParams p) {
+  using C = BwdCfg<D>;
+  constexpr int NQ = C::NQ;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  uint8_t* sK = smem;
+  uint8_t* sV = sK + C::TILE_BYTES;
+  uint8_t* sQ = sV + C::TILE_BYTES;                 // NQ tiles
+  uint8_t* sdO = sQ + NQ * C::TILE_BYTES;           // NQ tiles
+  uint8_t* sdS = sdO + NQ * C::TILE_BYTES;          // 128 x 128 bf16, two 64-column atoms
+  __shared__ BwdShared sh;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  // the 128-byte-swizzled operand tiles need 1024-byte aligned shared memory
+  if (smem_u32(smem) & 1023u) {
+    if (tid == 0 && p.err) atomicCAS(p.err, 0u, static_cast<uint32_t>(MALA_ERR_UNSUPPORTED));
+    return;
+  }
+  if (tid == 0) {
+    mbar_init(&sh.kv_full, 1);
+    mbar_init(&sh.kv_empty, 1);
+    for (int s = 0; s < NQ; ++s) {
+      mbar_init(&sh.q_full[s], 1);
+      mbar_init(&sh.q_empty[s], 1);
+    }
+    mbar_init(&sh.s_full, 1);
+    mbar_init(&sh.p_full, 256);
+    mbar_init(&sh.dp_full, 1);
+    mbar_init(&sh.ds_full, 256);
+    mbar_init(&sh.dq_full, 1);
+    mbar_init(&sh.dq_empty, 128);
+    mbar_init(&sh.acc_full, 1);
+    mbar_init(&sh.acc_empty, 128);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&sh.sched_full[s], 1);
+      mbar_init(&sh.sched_empty[s], 1 + 256 + 128);
+    }
+    mbar_init(&sh.final_bar, 1);
+    sh.abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&sh.tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tb = sh.tmem_base;
+  const uint32_t tS = tb, tdP = tb + 128, tdV = tb + 256, tdK = tb + 256 + D;
+  const AbortState ast{&sh.abort_flag, p.err, p.budget_ns, 0x200u};
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      tma_prefetch_desc(&tmdO);
+      uint32_t c = 0, nu = 0;
+      bool ok = true;
+      for (uint32_t k = 0; ok; ++k) {
+        const int ring = k & 1;
+        if (k >= 2 && !(ok = mbar_wait(&sh.sched_empty[ring], ((k >> 1) - 1) & 1, ast, 1))) break;
+        const int u = static_cast<int>(atomicAdd(p.sched, 1u));
+        sh.sched_ring[ring] = u;
+        mbar_arrive(&sh.sched_full[ring]);
+        if (u >= p.n_units) break;
+        const BUnit w = decode_bunit(p, u);
+        if (nu > 0 && !(ok = mbar_wait(&sh.kv_empty, (nu - 1) & 1, ast, 2))) break;
+        mbar_arrive_expect_tx(&sh.kv_full, 2 * C::TILE_BYTES);
+        for (int x = 0; x < C::BOXES; ++x) {
+          tma_load_4d(sK + x * 16384, &tmK, &sh.kv_full, x * 64, w.g, w.j * kTile, w.b);
+          tma_load_4d(sV + x * 16384, &tmV, &sh.kv_full, x * 64, w.g, w.j * kTile, w.b);
+        }
+        ++nu;
+        for (int n = 0; n < w.ntiles && ok; ++n, ++c) {
+          int h, i;
+          tile_hi(p, w, n, h, i);
+          const int st = c % NQ;
+          if (c >= NQ && !(ok = mbar_wait(&sh.q_empty[st], ((c / NQ) - 1) & 1, ast, 3))) break;
+          mbar_arrive_expect_tx(&sh.q_full[st], 2 * C::TILE_BYTES);
+          for (int x = 0; x < C::BOXES; ++x) {
+            tma_load_4d(sQ + st * C::TILE_BYTES + x * 16384, &tmQ, &sh.q_full[st], x * 64, h,
+                        i * kTile, w.b);
+            tma_load_4d(sdO + st * C::TILE_BYTES + x * 16384, &tmdO, &sh.q_full[st], x * 64, h,
+                        i * kTile, w.b);
+          }
+        }
+      }
+      if (!ok) {
+        AbortState drain = ast;
+        uint32_t zero = 0;
+        drain.flag = &zero;
+        drain.budget_ns = 200000000ull;
+        if (nu > 0) mbar_wait(&sh.kv_full, (nu - 1) & 1, drain, 4);
+        for (uint32_t cc = (c > NQ ? c - NQ : 0); cc < c; ++cc)
+          mbar_wait(&sh.q_full[cc % NQ], (cc / NQ) & 1, drain, 4);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t id_s = idesc_bf16(128, 128, 0, 0);    // S^T, dP^T
+      constexpr uint32_t id_acc = idesc_bf16(128, D, 0, 1);    // dV (TS), dK (SS)
+      constexpr uint32_t id_dq = idesc_bf16(128, D, 1, 1);     // dQ = dS K_j
+      const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), adS = smem_u32(sdS);
+      uint32_t c = 0, nu = 0, ntile = 0, nret = 0;  // tiles / retained tiles (all units)
+      bool acc_waited = true;  // acc_empty of the previous unit already observed
+      bool ok = true;
+      for (uint32_t k = 0; ok; ++k) {
+        const int ring = k & 1;
+        if (!(ok = mbar_wait(&sh.sched_full[ring], (k >> 1) & 1, ast, 10))) break;
+        const int u = sh.sched_ring[ring];
+        mbar_arrive(&sh.sched_empty[ring]);
+        if (u >= p.n_units) break;
+        const BUnit w = decode_bunit(p, u);
+        if (!(ok = mbar_wait(&sh.kv_full, nu & 1, ast, 11))) break;
+        bool acc_started = false;
+        acc_waited = (nu == 0);
+        auto issue_s = [&](uint32_t cc) {
+          const uint32_t aQ = smem_u32(sQ + (cc % NQ) * C::TILE_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+            umma_ss(tS, sdesc_sw128(aK + off, 16, 1024), sdesc_sw128(aQ + off, 16, 1024), id_s,
+                    kk > 0);
+          }
+          umma_commit(&sh.s_full);
+        };
+        // prologue: S^T of the first tile
+        if (!(ok = mbar_wait(&sh.q_full[c % NQ], (c / NQ) & 1, ast, 12))) break;
+        tc_fence_after();
+        issue_s(c);
+        for (int n = 0; n < w.ntiles && ok; ++n, ++c, ++ntile) {
+          const int st = c % NQ;
+          const uint32_t aQ = smem_u32(sQ + st * C::TILE_BYTES);
+          const uint32_t adO = smem_u32(sdO + st * C::TILE_BYTES);
+          if (!(ok = mbar_wait(&sh.p_full, ntile & 1, ast, 13))) break;
+          tc_fence_after();
+          const bool keep = sh.dec != 0;
+          if (keep) {
+            // dP^T reuses the columns of the previous dQ tile: wait for its drain
+            if (ntile > 0 && !(ok = mbar_wait(&sh.dq_empty, (ntile - 1) & 1, ast, 14))) break;
+            // first accumulation of the unit overwrites dK / dV: previous epilogue done
+            if (!acc_waited && !(ok = acc_waited = mbar_wait(&sh.acc_empty, (nu - 1) & 1, ast, 15)))
+              break;
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+              umma_ss(tdP, sdesc_sw128(aV + off, 16, 1024), sdesc_sw128(adO + off, 16, 1024),
+                      id_s, kk > 0);
+            }
+            umma_commit(&sh.dp_full);
+            // dV += P^T dO (P^T bf16 in TMEM columns [0, 64))
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+              umma_ts(tdV, tS + kk * 8, sdesc_sw128(adO + kk * 2048, 16384, 1024), id_acc,
+                      (acc_started || kk > 0) ? 1u : 0u);
+          }
+          // next tile's S^T (after dV has consumed P^T from the same columns)
+          if (n + 1 < w.ntiles) {
+            const uint32_t c1 = c + 1;
+            if (!(ok = mbar_wait(&sh.q_full[c1 % NQ], (c1 / NQ) & 1, ast, 16))) break;
+            tc_fence_after();
+            issue_s(c1);
+          }
+          if (keep) {
+            if (!(ok = mbar_wait(&sh.ds_full, nret & 1, ast, 17))) break;
+            tc_fence_after();
+            // dK += dS^T Q_i  (A = dS^T K-major, B = Q_i MN-major)
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+              const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+              umma_ss(tdK, sdesc_sw128(adS + off, 16, 1024),
+                      sdesc_sw128(aQ + kk * 2048, 16384, 1024), id_acc,
+                      (acc_started || kk > 0) ? 1u : 0u);
+            }
+            // dQ_i = dS K_j  (A = dS^T read MN-major, B = K_j MN-major) into dP^T columns
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+              umma_ss(tdP, sdesc_sw128(adS + kk * 2048, 16384, 1024),
+                      sdesc_sw128(aK + kk * 2048, 16384, 1024), id_dq, kk > 0);
+            acc_started = true;
+            ++nret;
+          }
+          // keep dq_full in lockstep with the drain (at most one phase ahead of it)
+          if (ntile > 0 && !(ok = mbar_wait(&sh.dq_empty, (ntile - 1) & 1, ast, 19))) break;
+          sh.dq_flag[ntile & 1] = keep ? 1u : 0u;
+          umma_commit(&sh.dq_full);
+          umma_commit(&sh.q_empty[st]);
+        }
+        if (!ok) break;
+        if (!acc_waited && !(ok = acc_waited = mbar_wait(&sh.acc_empty, (nu - 1) & 1, ast, 15)))
+          break;
+        sh.acc_valid = acc_started ? 1u : 0u;
+        umma_commit(&sh.acc_full);
+        umma_commit(&sh.kv_empty);
+        ++nu;
+      }
+      umma_commit(&sh.final_bar);
+      AbortState fin = ast;
+      uint32_t zero = 0;
+      fin.flag = &zero;
+      mbar_wait(&sh.final_bar, 0, fin, 18);
+    }
+  } else if (warp >= 4 && warp < 12) {
+    // ------------------------------------------------------------------ softmax
+    const int wg = (warp - 4) >> 2;         // query-column half
+    const int wq = warp & 3;
+    const int r = wq * 32 + lane;           // key row within the tile / TMEM lane
+    const int tw = tid - 128 - 128 * wg;    // 0..127 within the warpgroup
+    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+    const float NEG_INF = -INFINITY;
+    uint32_t ntile = 0, nret = 0;
+    bool ok = true;
+    uint8_t* dsrow_base = sdS + wg * 16384;  // this warpgroup's 64-column atom
+    for (uint32_t k = 0; ok; ++k) {
+      const int ring = k & 1;
+      const bool got = mbar_wait(&sh.sched_full[ring], (k >> 1) & 1, ast, 20);
+      if (named_bar_or(1, 256, !got) || *ast.flag) { ok = false; break; }
+      const int u = sh.sched_ring[ring];
+      mbar_arrive(&sh.sched_empty[ring]);
+      if (u >= p.n_units) break;
+      const BUnit w = decode_bunit(p, u);
+      const int krow = w.j * kTile + r;
+      const bool kvalid = krow < p.L;
+      for (int n = 0; n < w.ntiles; ++n, ++ntile) {
+        int h, i;
+        tile_hi(p, w, n, h, i);
+        // per-column constants of this tile (warpgroup-private buffers)
+        named_bar_sync(2 + wg, 128);  // previous tile's readers are done
+        if (tw < 64) {
+          const int q = i * kTile + wg * 64 + tw;
+          float c2 = INFINITY, l2 = 0.f, ds = 0.f;
+          if (q < p.L) {
+            const size_t idx = (static_cast<size_t>(w.b) * p.H + h) * p.L + q;
+            l2 = p.LSE[idx] * kLog2e;
+            ds = p.Dsum[idx];
+            c2 = kScreen ? l2 + (p.log2_tau - __log2f(static_cast<float>(q + 1))) : NEG_INF;
+          }
+          sh.c2[wg][tw] = c2;
+          sh.lse2[wg][tw] = l2;
+          sh.dsum[wg][tw] = ds;
+        }
+        named_bar_sync(2 + wg, 128);
+        const bool got = mbar_wait(&sh.s_full, ntile & 1, ast, 21);
+        tc_fence_after();
+        uint32_t v[2][32];
+        if (__all_sync(0xffffffffu, got)) {
+          tmem_ld32(tS + lane_off + wg * 64, v[0]);
+          tmem_ld32(tS + lane_off + wg * 64 + 32, v[1]);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int a = 0; a < 2; ++a)
+#pragma unroll
+            for (int e = 0; e < 32; ++e) v[a][e] = 0xff800000u;
+        }
+        // legal entries: key row valid, query q < L, and q >= k on the diagonal block
+        const int qlo = (i == w.j) ? (r - wg * 64) : -1;  // local column must be >= qlo
+        float ymax = NEG_INF;
+#pragma unroll
+        for (int a = 0; a < 2; ++a)
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const int cl = a * 32 + e;
+            float x = __uint_as_float(v[a][e]) * p.scale_log2;
+            const bool legal = kvalid && cl >= qlo && sh.c2[wg][cl] != INFINITY;
+            x = legal ? x : NEG_INF;
+            v[a][e] = __float_as_uint(x);
+            if (kScreen) ymax = fmaxf(ymax, x - sh.c2[wg][cl]);
+          }
+        bool keep = true;
+        if (kScreen) keep = named_bar_or(1, 256, ymax >= 0.f);
+        else named_bar_sync(1, 256);  // every S^T load done before P overwrites it
+        if (*ast.flag) { ok = false; break; }
+        if (p.tile_mask && tid == 128)
+          p.tile_mask[((static_cast<size_t>(w.b) * p.H + h) * p.T + i) * p.T + w.j] = keep ? 1 : 0;
+        if (!keep) {
+          if (tid == 128) sh.dec = 0;
+          tc_fence_before();
+          mbar_arrive(&sh.p_full);
+          continue;
+        }
+        // P^T = exp2(x - LSE2) -> bf16 pairs into TMEM columns [32 wg, 32 wg + 32)
+        float pf[64];
+#pragma unroll
+        for (int a = 0; a < 2; ++a) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int c0 = a * 32 + 2 * e;
+            const float p0 = fast_exp2(__uint_as_float(v[a][2 * e]) - sh.lse2[wg][c0]);
+            const float p1 = fast_exp2(__uint_as_float(v[a][2 * e + 1]) - sh.lse2[wg][c0 + 1]);
+            pf[c0] = p0;
+            pf[c0 + 1] = p1;
+            pk[e] = pack_bf16(p0, p1);
+          }
+          tmem_st16(tS + lane_off + wg * 32 + a * 16, pk);
+        }
+        tmem_wait_st();
+        if (tid == 128) sh.dec = 1;
+        tc_fence_before();
+        mbar_arrive(&sh.p_full);
+        // dS^T = P^T o (dP^T - D) * scale -> bf16, swizzled K-major rows in shared memory
+        const bool dp_ok = mbar_wait(&sh.dp_full, nret & 1, ast, 22);
+        ++nret;
+        // the dS^T buffer is free once the previous tile's dK / dQ MMAs completed
+        bool buf_ok = true;
+        if (ntile > 0) buf_ok = mbar_wait(&sh.dq_full, (ntile - 1) & 1, ast, 23);
+        tc_fence_after();
+        if (__all_sync(0xffffffffu, dp_ok && buf_ok)) {
+#pragma unroll
+          for (int a = 0; a < 2; ++a) {
+            uint32_t dp[32];
+            tmem_ld32(tdP + lane_off + wg * 64 + a * 32, dp);
+            tmem_wait_ld();
+#pragma unroll
+            for (int ch = 0; ch < 4; ++ch) {  // 4 chunks of 8 columns = 16 bytes
+              uint32_t pk[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const int c0 = a * 32 + ch * 8 + 2 * e;
+                const float d0 = pf[c0] * (__uint_as_float(dp[ch * 8 + 2 * e]) - sh.dsum[wg][c0]);
+                const float d1 =
+                    pf[c0 + 1] * (__uint_as_float(dp[ch * 8 + 2 * e + 1]) - sh.dsum[wg][c0 + 1]);
+                pk[e] = pack_bf16(d0 * p.scale, d1 * p.scale);
+              }
+              *reinterpret_cast<uint4*>(dsrow_base + sw128_offset(r, a * 4 + ch)) =
+                  make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            }
+          }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(&sh.ds_full);
+      }
+    }
+  } else if (warp >= 12) {
+    // ------------------------------------------------------------------ dQ drain + dK/dV epilogue
+    const int wq = warp & 3;
+    const int r = wq * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+    uint32_t ntile = 0, nu = 0;
+    bool ok = true;
+    for (uint32_t k = 0; ok; ++k) {
+      const int ring = k & 1;
+      const bool got = mbar_wait(&sh.sched_full[ring], (k >> 1) & 1, ast, 30);
+      if (named_bar_or(4, 128, !got) || *ast.flag) { ok = false; break; }
+      const int u = sh.sched_ring[ring];
+      mbar_arrive(&sh.sched_empty[ring]);
+      if (u >= p.n_units) break;
+      const BUnit w = decode_bunit(p, u);
+      for (int n = 0; n < w.ntiles; ++n, ++ntile) {
+        int h, i;
+        tile_hi(p, w, n, h, i);
+        const bool got_dq = __all_sync(0xffffffffu, mbar_wait(&sh.dq_full, ntile & 1, ast, 31));
+        tc_fence_after();
+        if (got_dq && sh.dq_flag[ntile & 1]) {
+          const int q = i * kTile + r;
+          float* dst = p.dQacc + ((static_cast<size_t>(w.b) * p.L + q) * p.H + h) * D;
+#pragma unroll
+          for (int a = 0; a < D / 32; ++a) {
+            uint32_t o[32];
+            tmem_ld32(tdP + lane_off + a * 32, o);
+            tmem_wait_ld();
+            if (q < p.L) {
+#pragma unroll
+              for (int e = 0; e < 8; ++e)
+                red_add_v4(dst + a * 32 + 4 * e, __uint_as_float(o[4 * e]),
+                           __uint_as_float(o[4 * e + 1]), __uint_as_float(o[4 * e + 2]),
+                           __uint_as_float(o[4 * e + 3]));
+            }
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(&sh.dq_empty);
+      }
+      // unit epilogue: dK, dV of key block j
+      const bool got_acc = __all_sync(0xffffffffu, mbar_wait(&sh.acc_full, nu & 1, ast, 32));
+      tc_fence_after();
+      const bool valid_acc = sh.acc_valid != 0;
+      const int krow = w.j * kTile + r;
+      // tcgen05.ld is warp-collective: every lane loads, only rows < L are stored
+      if (got_acc) {
+        const bool store = krow < p.L;
+        const size_t base = ((static_cast<size_t>(w.b) * p.L + (store ? krow : 0)) * p.Hkv + w.g) * D;
+#pragma unroll
+        for (int which = 0; which < 2; ++which) {
+          __nv_bfloat16* dst = (which == 0 ? p.dV : p.dK) + base;
+          const uint32_t src = (which == 0 ? tdV : tdK) + lane_off;
+#pragma unroll
+          for (int a = 0; a < D / 32; ++a) {
+            uint32_t o[32];
+            tmem_ld32(src + a * 32, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e8 = 0; e8 < 4; ++e8) {
+              uint4 pk;
+              const float* f = reinterpret_cast<const float*>(o) + e8 * 8;
+              if (valid_acc) {
+                pk.x = pack_bf16(f[0], f[1]);
+                pk.y = pack_bf16(f[2], f[3]);
+                pk.z = pack_bf16(f[4], f[5]);
+                pk.w = pack_bf16(f[6], f[7]);
+              } else {
+                pk = make_uint4(0u, 0u, 0u, 0u);
+              }
+              if (store) *reinterpret_cast<uint4*>(dst + a * 32 + e8 * 8) = pk;
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&sh.acc_empty);
+      ++nu;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tb, 512);
+}
+
+// D_q = <O_q, dO_q> and zeroing of the dQ accumulator; one warp per (b, q, h) row.
+template <int D>
+__global__ void __launch_bounds__(256) mala_bwd_prep(const __nv_bfloat16* __restrict__ O,
+                                                     const __nv_bfloat16* __restrict__ dO,
+                                                     float* __restrict__ Dsum,
+                                                     float* __restrict__ dQacc, int B, int L,
+                                                     int H) {
+  const long long row = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= static_cast<long long>(B) * L * H) return;
+  constexpr int PER = D / 32;  // elements per lane (2 or 4)
+  const __nv_bfloat16* o = O + row * D + lane * PER;
+  const __nv_bfloat16* g = dO + row * D + lane * PER;
+  float s = 0.f;
+#pragma unroll
+  for (int e = 0; e < PER; e += 2) {
+    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(o + e));
+    const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(g + e));
+    s += a.x * b.x + a.y * b.y;
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+  float* z = dQacc + row * D + lane * PER;
+#pragma unroll
+  for (int e = 0; e < PER; ++e) z[e] = 0.f;
+  if (lane == 0) {
+    const int h = static_cast<int>(row % H);
+    const long long bq = row / H;
+    const int q = static_cast<int>(bq % L);
+    const int b = static_cast<int>(bq / L);
+    Dsum[(static_cast<long long>(b) * H + h) * L + q] = s;
+  }
+}
+
+__global__ void __launch_bounds__(256) mala_bwd_dq(const float* __restrict__ acc,
+                                                   __nv_bfloat16* __restrict__ dQ, long long n4) {
+  const long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= n4) return;
+  const float4 v = reinterpret_cast<const float4*>(acc)[i];
+  uint2 pk;
+  pk.x = pack_bf16(v.x, v.y);
+  pk.y = pack_bf16(v.z, v.w);
+  reinterpret_cast<uint2*>(dQ)[i] = pk;
+}
+
+}  // namespace
+
 size_t bwd_workspace_bytes(int B, int H, int Hkv, int L, int d, int dtype) {
   (void)Hkv; (void)dtype;
-  return kWorkspaceHeader + (size_t)B * L * H * d * 4 + (size_t)B * H * L * 4;
+  const size_t acc = static_cast<size_t>(B) * L * H * d * sizeof(float);
+  const size_t dsum = static_cast<size_t>(B) * H * L * sizeof(float);
+  return kWorkspaceHeader + ((acc + 255) / 256) * 256 + ((dsum + 255) / 256) * 256;
 }
-mala_status bwd_dispatch(const void*, const void*, const void*, const void*, const float*,
-                         const void*, void*, void*, void*, int, int, int, int, int, int, float,
-                         float, unsigned, uint8_t*, uint8_t*, uint64_t, cudaStream_t) {
-  return MALA_ERR_UNSUPPORTED;
+
+mala_status fp32_bwd(const float* Q, const float* K, const float* V, const float* O,
+                     const float* LSE, const float* dO, float* dQ, float* dK, float* dV, int B,
+                     int H, int Hkv, int L, int d, float scale, float tau, bool screen,
+                     uint8_t* ws, uint8_t* tile_mask, cudaStream_t stream);
+
+template <int D, bool kScreen>
+static cudaError_t launch_bwd_main(const CUtensorMap& tq, const CUtensorMap& tk,
+                                   const CUtensorMap& tv, const CUtensorMap& tdo,
+                                   const BwdParams& p, int grid, cudaStream_t stream) {
+  auto kern = mala_bwd_kernel<D, kScreen>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       BwdCfg<D>::SMEM);
+  if (e != cudaSuccess) return e;
+  kern<<<grid, kBwdThreads, BwdCfg<D>::SMEM, stream>>>(tq, tk, tv, tdo, p);
+  return cudaGetLastError();
 }
+
+mala_status bwd_dispatch(const void* Q, const void* K, const void* V, const void* O,
+                         const float* LSE, const void* dO, void* dQ, void* dK, void* dV, int B,
+                         int H, int Hkv, int L, int d, int dtype, float scale, float tau,
+                         unsigned flags, uint8_t* ws, uint8_t* tile_mask, uint64_t budget_ns,
+                         cudaStream_t stream) {
+  const bool screen = (tau > 0.f) || (flags & MALA_FLAG_ALWAYS_TEST);
+  if (dtype == MALA_FP32)
+    return fp32_bwd(static_cast<const float*>(Q), static_cast<const float*>(K),
+                    static_cast<const float*>(V), static_cast<const float*>(O), LSE,
+                    static_cast<const float*>(dO), static_cast<float*>(dQ),
+                    static_cast<float*>(dK), static_cast<float*>(dV), B, H, Hkv, L, d, scale,
+                    tau, screen, ws, tile_mask, stream);
+  const int T = (L + kTile - 1) / kTile;
+  CUtensorMap tq, tk, tv, tdo;
+  if (!make_tile_map(&tq, Q, d, H, L, B) || !make_tile_map(&tk, K, d, Hkv, L, B) ||
+      !make_tile_map(&tv, V, d, Hkv, L, B) || !make_tile_map(&tdo, dO, d, H, L, B))
+    return MALA_ERR_CUDA;
+  uint32_t* hdr = reinterpret_cast<uint32_t*>(ws);
+  const size_t acc_bytes = static_cast<size_t>(B) * L * H * d * sizeof(float);
+  float* dQacc = reinterpret_cast<float*>(ws + kWorkspaceHeader);
+  float* Dsum = reinterpret_cast<float*>(ws + kWorkspaceHeader + ((acc_bytes + 255) / 256) * 256);
+  if (cudaMemsetAsync(hdr + kHdrSched0, 0, 3 * sizeof(uint32_t), stream) != cudaSuccess)
+    return MALA_ERR_CUDA;
+  const long long rows = static_cast<long long>(B) * L * H;
+  const unsigned prep_blocks = static_cast<unsigned>((rows + 7) / 8);
+  if (d == 128)
+    mala_bwd_prep<128><<<prep_blocks, 256, 0, stream>>>(
+        static_cast<const __nv_bfloat16*>(O), static_cast<const __nv_bfloat16*>(dO), Dsum, dQacc,
+        B, L, H);
+  else
+    mala_bwd_prep<64><<<prep_blocks, 256, 0, stream>>>(
+        static_cast<const __nv_bfloat16*>(O), static_cast<const __nv_bfloat16*>(dO), Dsum, dQacc,
+        B, L, H);
+  if (cudaGetLastError() != cudaSuccess) return MALA_ERR_CUDA;
+  BwdParams p;
+  p.B = B; p.H = H; p.Hkv = Hkv; p.L = L; p.T = T; p.G = H / Hkv;
+  p.n_units = T * B * Hkv;
+  p.scale = scale;
+  p.scale_log2 = scale * kLog2e;
+  p.log2_tau = (tau > 0.f) ? std::log2(tau) : -INFINITY;
+  p.LSE = LSE; p.Dsum = Dsum; p.dQacc = dQacc;
+  p.dK = static_cast<__nv_bfloat16*>(dK);
+  p.dV = static_cast<__nv_bfloat16*>(dV);
+  p.tile_mask = tile_mask;
+  p.err = hdr + kHdrError;
+  p.sched = hdr + kHdrSched0;
+  p.budget_ns = budget_ns;
+  const int grid = p.n_units < sm_count() ? p.n_units : sm_count();
+  cudaError_t e;
+  if (d == 128)
+    e = screen ? launch_bwd_main<128, true>(tq, tk, tv, tdo, p, grid, stream)
+               : launch_bwd_main<128, false>(tq, tk, tv, tdo, p, grid, stream);
+  else
+    e = screen ? launch_bwd_main<64, true>(tq, tk, tv, tdo, p, grid, stream)
+               : launch_bwd_main<64, false>(tq, tk, tv, tdo, p, grid, stream);
+  if (e != cudaSuccess) return MALA_ERR_CUDA;
+  const long long n4 = rows * d / 4;
+  mala_bwd_dq<<<static_cast<unsigned>((n4 + 255) / 256), 256, 0, stream>>>(
+      dQacc, static_cast<__nv_bfloat16*>(dQ), n4);
+  return cudaGetLastError() == cudaSuccess ? MALA_OK : MALA_ERR_CUDA;
+}
+
 }  // namespace mala

@@ -13,3 +13,10 @@ mala_status fp32_decode(const float*, const float*, const float*, float*, float*
   return MALA_ERR_UNSUPPORTED;
 }
 }  // namespace mala
+namespace mala {
+mala_status fp32_bwd(const float*, const float*, const float*, const float*, const float*,
+                     const float*, float*, float*, float*, int, int, int, int, int, float, float,
+                     bool, uint8_t*, uint8_t*, cudaStream_t) {
+  return MALA_ERR_UNSUPPORTED;
+}
+}  // namespace mala
