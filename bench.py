@@ -1,0 +1,492 @@
+#!/usr/bin/env python3
+"""Benchmark of the MALA hot path on B200: training forward + backward at 32K and split-KV
+decode at 128K, through the library's C ABI.
+
+One step = mala_fwd + mala_bwd on the 32K training workload (B=1, H=32, H_kv=8,
+L=32768, d=128, bf16, sink + local-band synthetic states, tau = 1) followed by one
+mala_decode on the 128K decode workload (B=4, H=32, H_kv=8, N_k=131072, d=128, planted
+keys, tau = 1).  The same steps are also timed at tau = 0 (the library's dense path).
+
+Usage:  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl mala|reference]
+Multi-GPU: launched by torch.distributed.run, one rank per GPU; every rank runs its own
+independent problem (different seeds) with no collective on the data path (weak
+scaling); timing is the max over ranks.  Prints one JSON line on rank 0.
+"""
+
+from __future__ import annotations
+
+import argparse
+import dataclasses
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from mass_adaptive_sparse_fwd_b200 import synth  # noqa: E402
+
+METRIC = "MALA fwd+bwd ms and TFLOPS at 32K, decode µs at 128K; % of bf16 tensor peak"
+TRAIN = "sinkband32k"
+DECODE = "decode128k"
+TAU = 1.0
+KERNELS_PER_STEP = 5  # fwd 1, bwd 3 (D preprocess, main, dQ convert), decode 1
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            pk = json.load(f)
+        return {"hbm_gbs": pk["hbm_gbs"], "bf16_tflops": pk["bf16_tflops"],
+                "bf16_tflops_sustained": pk["bf16_tflops_sustained"], "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+# ----------------------------------------------------------------------------- dist
+
+
+class Dist:
+    def __init__(self):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+        self.pg = None
+
+    def init(self, backend: str):
+        if self.world > 1:
+            import datetime
+
+            import torch.distributed as dist
+
+            os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+            dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+            self.pg = dist
+        return self
+
+    def barrier(self):
+        if self.pg is not None:
+            if self.pg.get_backend() == "nccl":
+                self.pg.barrier(device_ids=[self.local_rank])
+            else:
+                self.pg.barrier()
+
+    def max(self, x: float, device="cpu") -> float:
+        if self.pg is None:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=device)
+        self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.pg is not None:
+            self.pg.destroy_process_group()
+
+
+def rank_workload(w: synth.Workload, rank: int) -> synth.Workload:
+    """Each rank gets an independent problem of the same shape (weak scaling)."""
+    return dataclasses.replace(w, seed=w.seed + 1000 * rank)
+
+
+# ----------------------------------------------------------------------------- work accounting
+
+
+def fwd_bwd_flops(w: synth.Workload, fwd_retained: float, bwd_retained: float):
+    """Executed and dense-equivalent FLOPs of one forward + backward (tile granular).
+    Forward: QK^T on every legal tile + PV on retained tiles; backward: QK^T recompute on
+    every legal tile + dP, dV, dK, dQ on retained tiles (Eq. (13)/(16) accounting)."""
+    T = math.ceil(w.L / 128)
+    legal = T * (T + 1) // 2 * w.B * w.H
+    per = 2.0 * w.d * 128 * 128
+    fwd_exec = per * legal * (1.0 + fwd_retained)
+    bwd_exec = per * legal * (1.0 + 4.0 * bwd_retained)
+    pairs = w.L * (w.L + 1) / 2 * w.B * w.H
+    return {"fwd_exec": fwd_exec, "bwd_exec": bwd_exec, "fwd_dense_eq": 4.0 * w.d * pairs,
+            "bwd_dense_eq": 10.0 * w.d * pairs, "legal_tiles": legal}
+
+
+def decode_bytes(w: synth.Workload, vtiles_loaded: int, S: int) -> float:
+    """Algorithmic HBM bytes of one decode call: all K, the V tiles some head of the
+    group retained, q / O and the split partials."""
+    kbytes = w.B * w.H_kv * w.L * w.d * 2
+    vbytes = vtiles_loaded * 128 * w.d * 2
+    qo = 2 * w.B * w.H * w.d * 2
+    part = 2 * w.B * w.H * S * (w.d + 1) * 4
+    return kbytes + vbytes + qo + part
+
+
+# ----------------------------------------------------------------------------- clocks
+
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.f,
+                stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.f.close()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 8:
+                    continue
+                try:
+                    sm.append(float(parts[0]))
+                    smax.append(float(parts[1]))
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[4:8]):
+                    if v.lower() == "active":
+                        reasons.add(n)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+
+
+def oracle_sample(wt: synth.Workload, wd: synth.Workload, train, dec, S: int,
+                  small: bool = False):
+    """Times the fp64 CPU oracle on a bounded sample of one step and extrapolates to the
+    full step by tile counts.  Returns (ms_per_full_step, seconds_spent, description)."""
+    import oracle
+
+    oracle.build()
+    T = wt.L // 128
+    if small:  # a few seconds: one reference-arm step
+        fwd_units = [(0, 0, T // 4)]
+        kv_units = [(0, wt.H_kv - 1, T - 6)]
+        q_units = [(0, 5, 15)]
+    else:      # about 10-30 s on a few cores: the cpu_baseline of the GPU arm
+        fwd_units = [(0, 0, T - 1), (0, wt.H // 2, T // 2)]
+        kv_units = [(0, wt.H_kv - 1, T - 24)]
+        q_units = [(0, 5, 23)]
+    t0 = time.perf_counter()
+    O, LSE, _, _ = oracle.mala_fwd(train["Q"], train["K"], train["V"], wt.scale, TAU,
+                                   units=fwd_units)
+    t1 = time.perf_counter()
+    # backward conditioned on the oracle's own rows where it has them, else a flat LSE
+    LSEc = np.where(np.isfinite(LSE), LSE, np.log(np.arange(1, wt.L + 1))[None, None, :])
+    Oc = np.where(np.isfinite(O), O, 0.0)
+    oracle.mala_bwd(train["Q"], train["K"], train["V"], Oc, LSEc, train["dO"], wt.scale, TAU,
+                    kv_units=kv_units, q_units=q_units)
+    t2 = time.perf_counter()
+    dunits = [(0, 0)]
+    oracle.mala_decode(dec["q"], dec["K"], dec["V"], wd.scale, TAU, S, units=dunits)
+    t3 = time.perf_counter()
+    G = wt.H // wt.H_kv
+    fwd_tiles = sum(i + 1 for _, _, i in fwd_units)
+    bwd_tiles = sum(G * (T - j) for _, _, j in kv_units) + sum(i + 1 for _, _, i in q_units)
+    legal = T * (T + 1) // 2 * wt.B * wt.H
+    full_ms = 1e3 * ((t1 - t0) / fwd_tiles * legal + (t2 - t1) / bwd_tiles * 2 * legal +
+                     (t3 - t2) / len(dunits) * wd.B * wd.H)
+    desc = (f"oracle fp64 on {fwd_units} forward query blocks, {kv_units} dK/dV key blocks, "
+            f"{q_units} dQ query blocks of {TRAIN} and {len(dunits)} of {wd.B * wd.H} decode "
+            f"rows of {DECODE}; extrapolated to the full step by tile / row counts")
+    return full_ms, t3 - t0, desc
+
+
+def omp_threads() -> int:
+    v = os.environ.get("OMP_NUM_THREADS")
+    return int(v) if v else (os.cpu_count() or 1)
+
+
+def run_reference(args, dist: Dist):
+    """Reference arm: the CPU oracle as it stands, each step a bounded sample."""
+    if dist.rank != 0:
+        return
+    wt, wd = synth.WORKLOADS[TRAIN], synth.WORKLOADS[DECODE]
+    train = synth.make_training(wt)
+    dec = synth.make_decode(wd)
+    S = 37
+    vals = []
+    for s in range(args.warmup + args.steps):
+        ms, spent, desc = oracle_sample(wt, wd, train, dec, S, small=True)
+        if s >= args.warmup:
+            vals.append(ms)
+    value = statistics.mean(vals)
+    cores = omp_threads()
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "ms",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": value, "higher_is_better": False, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": f"{TRAIN} fwd+bwd + {DECODE} decode", "tau": TAU},
+            "cpu_baseline": {"value": value, "unit": "ms", "cores": cores, "kind": "oracle",
+                             "sample": desc},
+            "e2e": {"value": value, "unit": "ms", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------- GPU arm
+
+
+def run_mala(args, dist: Dist):
+    from mass_adaptive_sparse_fwd_b200 import mala
+
+    dev = torch.device("cuda", dist.local_rank)
+    torch.cuda.set_device(dev)
+    peaks = _peaks()
+    wt = rank_workload(synth.WORKLOADS[TRAIN], dist.rank)
+    wd = rank_workload(synth.WORKLOADS[DECODE], dist.rank)
+    train = synth.make_training(wt)
+    dec = synth.make_decode(wd)
+    bf = lambda x: torch.from_numpy(x).to(dev).to(torch.bfloat16)
+    Q, K, V, dO = (bf(train[k]) for k in ("Q", "K", "V", "dO"))
+    q, Kc, Vc = (bf(dec[k]) for k in ("q", "K", "V"))
+    B, L, H, d = Q.shape
+    Hkv = K.shape[2]
+    S = mala.decode_num_splits(wd.B, wd.H, wd.H_kv, wd.L)
+    O = torch.empty_like(Q)
+    LSE = torch.empty((B, H, L), dtype=torch.float32, device=dev)
+    dQ, dK, dV = torch.empty_like(Q), torch.empty_like(K), torch.empty_like(V)
+    Od = torch.empty_like(q)
+    LSEd = torch.empty((wd.B, wd.H), dtype=torch.float32, device=dev)
+    wsf = mala.alloc_workspace(mala.fwd_workspace_bytes(B, H, Hkv, L, d), dev)
+    wsb = mala.alloc_workspace(mala.bwd_workspace_bytes(B, H, Hkv, L, d), dev)
+    wsd = mala.alloc_workspace(mala.decode_workspace_bytes(wd.B, wd.H, wd.H_kv, wd.L, d, 0, S),
+                               dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(tau, ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        mala.mala_fwd(Q, K, V, wt.scale, tau, O=O, LSE=LSE, workspace=wsf)
+        if ev is not None:
+            ev[1].record(stream)
+        mala.mala_bwd(Q, K, V, O, LSE, dO, wt.scale, tau, dQ=dQ, dK=dK, dV=dV, workspace=wsb)
+        if ev is not None:
+            ev[2].record(stream)
+        mala.mala_decode(q, Kc, Vc, wd.scale, tau, num_splits=S, O=Od, LSE=LSEd, workspace=wsd)
+        if ev is not None:
+            ev[3].record(stream)
+
+    def timed(tau, clocks=None):
+        for _ in range(args.warmup):
+            step(tau)
+        torch.cuda.synchronize(dev)
+        dist.barrier()
+        torch.cuda.synchronize(dev)
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+        if clocks:
+            clocks.start()
+        start = torch.cuda.Event(enable_timing=True)
+        end = torch.cuda.Event(enable_timing=True)
+        start.record(stream)
+        for k in range(args.steps):
+            step(tau, evs[k])
+        end.record(stream)
+        torch.cuda.synchronize(dev)
+        dist.barrier()
+        torch.cuda.synchronize(dev)
+        clk = clocks.stop() if clocks else None
+        total = start.elapsed_time(end) / args.steps
+        fwd = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+        bwd = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+        dcd = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
+        for ws in (wsf, wsb, wsd):
+            err = mala.read_device_error(ws)
+            if err:
+                raise RuntimeError(f"device error word 0x{err:x}")
+        return {"step_ms": total, "fwd_ms": fwd, "bwd_ms": bwd, "decode_ms": dcd, "clocks": clk}
+
+    clocks = ClockSampler(torch.cuda.current_device()) if dist.rank == 0 else None
+    res = timed(TAU, clocks)
+    res0 = timed(0.0)
+    # max over ranks of every figure (device timing)
+    for r in (res, res0):
+        for k in ("step_ms", "fwd_ms", "bwd_ms", "decode_ms"):
+            r[k] = dist.max(r[k], device=dev)
+
+    # retained work (one masked call of each operator, outside the timed region)
+    T = mala.n_tiles(L)
+    fmask = torch.zeros((B, H, T, T), dtype=torch.uint8, device=dev)
+    bmask = torch.zeros((B, H, T, T), dtype=torch.uint8, device=dev)
+    dmask = torch.zeros((wd.B, wd.H, mala.n_tiles(wd.L)), dtype=torch.uint8, device=dev)
+    mala.mala_fwd(Q, K, V, wt.scale, TAU, O=O, LSE=LSE, workspace=wsf, tile_mask=fmask)
+    mala.mala_bwd(Q, K, V, O, LSE, dO, wt.scale, TAU, dQ=dQ, dK=dK, dV=dV, workspace=wsb,
+                  tile_mask=bmask)
+    mala.mala_decode(q, Kc, Vc, wd.scale, TAU, num_splits=S, O=Od, LSE=LSEd, workspace=wsd,
+                     tile_mask=dmask)
+    torch.cuda.synchronize(dev)
+    legal = torch.ones(T, T, dtype=torch.bool, device=dev).tril()
+    fret = float(fmask[:, :, legal].float().mean())
+    bret = float(bmask[:, :, legal].float().mean())
+    G = wd.H // wd.H_kv
+    group_keep = dmask.view(wd.B, wd.H_kv, G, -1).amax(dim=2)
+    vtiles = int(group_keep.sum())
+    dret = float(dmask.float().mean())
+    # slots per query (M1): retained tiles contribute 128 key slots to each of their rows
+    fl = fwd_bwd_flops(wt, fret, bret)
+    dense_fl = fwd_bwd_flops(wt, 1.0, 1.0)
+    step_fb = res["fwd_ms"] + res["bwd_ms"]
+    dense_fb = res0["fwd_ms"] + res0["bwd_ms"]
+    exec_tf = (fl["fwd_exec"] + fl["bwd_exec"]) / (step_fb * 1e-3) / 1e12
+    deq_tf = (fl["fwd_dense_eq"] + fl["bwd_dense_eq"]) / (step_fb * 1e-3) / 1e12
+    dense_exec_tf = (dense_fl["fwd_exec"] + dense_fl["bwd_exec"]) / (dense_fb * 1e-3) / 1e12
+    dbytes = decode_bytes(wd, vtiles, S)
+    dbytes0 = decode_bytes(wd, wd.B * wd.H_kv * mala.n_tiles(wd.L), S)
+    dec_gbs = dbytes / (res["decode_ms"] * 1e-3) / 1e9
+    dec_gbs0 = dbytes0 / (res0["decode_ms"] * 1e-3) / 1e9
+
+    # roofline of the dominant kernel: the backward call (timed span includes its small
+    # D-preprocess and dQ-convert kernels; the main kernel dominates the share)
+    peak = peaks["bf16_tflops_sustained"]
+    bwd_tf = fl["bwd_exec"] / (res["bwd_ms"] * 1e-3) / 1e12
+    traffic = None
+    prof = os.path.join(ROOT, "profiles", "roofline_traffic.json")
+    if os.path.exists(prof):
+        with open(prof) as f:
+            tr = json.load(f)
+        traffic = tr.get("mala_bwd_kernel_bytes_per_launch")
+
+    # end to end through the C ABI with host buffers (pinned), copies in the timed region
+    e2e = None
+    if not args.no_e2e:
+        host_in = {k: torch.from_numpy(train[k]).to(torch.bfloat16).pin_memory()
+                   for k in ("Q", "K", "V", "dO")}
+        host_q = torch.from_numpy(dec["q"]).to(torch.bfloat16).pin_memory()
+        host_out = {n: torch.empty(t.shape, dtype=t.dtype).pin_memory()
+                    for n, t in (("O", O), ("LSE", LSE), ("dQ", dQ), ("dK", dK), ("dV", dV),
+                                 ("Od", Od), ("LSEd", LSEd))}
+        dev_out = {"O": O, "LSE": LSE, "dQ": dQ, "dK": dK, "dV": dV, "Od": Od, "LSEd": LSEd}
+        dev_in = {"Q": Q, "K": K, "V": V, "dO": dO}
+
+        def e2e_step():
+            for k, t in host_in.items():
+                dev_in[k].copy_(t, non_blocking=True)
+            q.copy_(host_q, non_blocking=True)
+            step(TAU)
+            for k, t in dev_out.items():
+                host_out[k].copy_(t, non_blocking=True)
+
+        for _ in range(args.warmup):
+            e2e_step()
+        torch.cuda.synchronize(dev)
+        dist.barrier()
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s0.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        s1.record(stream)
+        torch.cuda.synchronize(dev)
+        dist.barrier()
+        e2e_ms = dist.max(s0.elapsed_time(s1) / args.steps, device=dev)
+        h2d = sum(t.numel() * t.element_size() for t in host_in.values()) + \
+            host_q.numel() * host_q.element_size()
+        d2h = sum(t.numel() * t.element_size() for t in host_out.values())
+        e2e = {"value": e2e_ms, "unit": "ms", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h,
+               "note": "fwd+bwd+decode step incl. host->device inputs (Q,K,V,dO,q; the KV "
+                       "cache is resident) and device->host outputs"}
+
+    cpu = None
+    if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
+        ms, spent, desc = oracle_sample(wt, wd, train, dec, S)
+        cpu = {"value": ms, "unit": "ms", "cores": omp_threads(), "kind": "oracle",
+               "sample": desc + f" ({spent:.1f} s of CPU time)"}
+
+    if dist.rank == 0:
+        clk = res["clocks"] or {}
+        line = {
+            "metric": METRIC, "value": step_fb, "unit": "ms", "n_gpus": dist.world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": res["step_ms"], "higher_is_better": False, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded generator; states stand in for real model states)",
+            "config": {"workload": f"{TRAIN} fwd+bwd (B=1,H=32,H_kv=8,L=32768,d=128) + "
+                                   f"{DECODE} decode (B=4,H=32,H_kv=8,N_k=131072,d=128)",
+                       "tau": TAU, "decode_splits": S,
+                       "l2": "inputs larger than L2 (Q 268 MB, dO 268 MB, KV cache 2.1 GB)",
+                       "parallelism": f"weak: {dist.world} independent problem(s), one per GPU"},
+            "fwd_ms": res["fwd_ms"], "bwd_ms": res["bwd_ms"], "decode_us": res["decode_ms"] * 1e3,
+            "tflops": {"executed": exec_tf, "dense_equivalent": deq_tf},
+            "pct_bf16_peak": {"executed": exec_tf / peak, "bwd_kernel": bwd_tf / peak,
+                              "peak_tflops": peak, "peak": peaks["source"] + " sustained"},
+            "retained": {"fwd_tiles": fret, "bwd_tiles": bret, "decode_tiles": dret,
+                         "decode_v_tiles": vtiles / (wd.B * wd.H_kv * mala.n_tiles(wd.L)),
+                         "fwd_slots_per_query": fret * (L + 128) / 2.0},
+            "decode_gbs": dec_gbs,
+            "dense_tau0": {"fwd_ms": res0["fwd_ms"], "bwd_ms": res0["bwd_ms"],
+                           "fwd_bwd_ms": dense_fb, "decode_us": res0["decode_ms"] * 1e3,
+                           "tflops": dense_exec_tf, "pct_bf16_peak": dense_exec_tf / peak,
+                           "decode_gbs": dec_gbs0},
+            "speedup_vs_tau0": {"fwd_bwd": dense_fb / step_fb,
+                                "decode": res0["decode_ms"] / res["decode_ms"]},
+            "roofline": {"bound": "tensor", "kernel": "mala_bwd (main kernel + 2 small kernels)",
+                         "achieved": bwd_tf, "peak": peak, "unit": "TFLOP/s",
+                         "frac": bwd_tf / peak, "traffic": traffic,
+                         "peak_source": peaks["source"] + " bf16 sustained"},
+            "decode_roofline": {"bound": "hbm", "achieved": dec_gbs, "peak": peaks["hbm_gbs"],
+                                "unit": "GB/s", "frac": dec_gbs / peaks["hbm_gbs"]},
+            "clocks": {"sm_mhz": clk.get("sm_mhz"), "sm_max_mhz": clk.get("sm_max_mhz"),
+                       "reasons": clk.get("reasons", [])},
+            "gpu_launches": KERNELS_PER_STEP * args.steps,
+            "e2e": e2e,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=("mala", "reference"), default="mala")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    dist = Dist()
+    if args.impl == "reference":
+        run_reference(args, dist)  # rank 0 only; no process group needed
+        return
+    dist.init("nccl")
+    try:
+        run_mala(args, dist)
+    finally:
+        dist.close()
+
+
+if __name__ == "__main__":
+    main()

@@ -174,6 +174,8 @@ mala_status mala_fwd(const void* Q, const void* K, const void* V, void* O, float
   if (d != 64 && d != 128) return MALA_ERR_UNSUPPORTED;
   if ((long long)B * L > (1ll << 31) || (long long)B * H * T > (1ll << 30))
     return MALA_ERR_UNSUPPORTED;
+  if (workspace && workspace_bytes < mala_fwd_workspace_bytes(B, H, H_kv, L, d, dtype))
+    return MALA_ERR_WORKSPACE;
   CUtensorMap tq, tk, tv;
   if (!make_tile_map(&tq, Q, d, H, L, B) || !make_tile_map(&tk, K, d, H_kv, L, B) ||
       !make_tile_map(&tv, V, d, H_kv, L, B))

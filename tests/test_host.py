@@ -1,0 +1,146 @@
+"""Host-side checks that need no GPU: the C ABI exports, argument validation (which
+returns before any CUDA call), workspace-size queries, the bench's accounting helpers and
+its multi-rank plumbing (world size 2 over gloo)."""
+
+import ctypes
+import os
+import re
+import subprocess
+import sys
+
+import numpy as np
+import pytest
+import torch
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    names = []
+    for h in os.listdir(os.path.join(ROOT, "include")):
+        if h.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", h)).read()
+            names += re.findall(r"^\s*(?:[\w\*]+\s+)+\**(mala_\w+)\s*\(", src, re.M)
+    return sorted(set(names))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from mass_adaptive_sparse_fwd_b200 import build
+
+    build.build_library()
+    from mass_adaptive_sparse_fwd_b200 import mala
+
+    return mala
+
+
+def test_header_declares_the_three_operators():
+    names = _declared_functions()
+    for n in ("mala_fwd", "mala_bwd", "mala_decode"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    so = ctypes.CDLL(lib._LIB_PATH)
+    for n in _declared_functions():
+        assert hasattr(so, n), n
+    out = subprocess.run(["nm", "-D", "--defined-only", lib._LIB_PATH], capture_output=True,
+                         text=True).stdout
+    for n in _declared_functions():
+        assert re.search(rf"\bT {n}\b", out), n
+
+
+def test_version_and_status_strings(lib):
+    L = lib.lib()
+    assert L.mala_version() == 100
+    assert L.mala_status_string(0) == b"ok"
+    assert L.mala_status_string(4) == b"device wait timed out"
+
+
+def test_invalid_arguments_are_rejected_before_any_launch(lib):
+    L = lib.lib()
+    p = ctypes.c_void_p(16 * 1024)  # never dereferenced: validation fails first
+    vp = lambda: p
+    # H not a multiple of H_kv
+    assert L.mala_fwd(vp(), vp(), vp(), vp(), vp(), 1, 6, 4, 128, 128, 0, 0.1, 1.0, 0, None, 0,
+                      None, None) == 1
+    # negative tau, non-finite scale, zero length
+    assert L.mala_fwd(vp(), vp(), vp(), vp(), vp(), 1, 4, 2, 128, 128, 0, 0.1, -1.0, 0, None, 0,
+                      None, None) == 1
+    assert L.mala_fwd(vp(), vp(), vp(), vp(), vp(), 1, 4, 2, 128, 128, 0, float("nan"), 1.0, 0,
+                      None, 0, None, None) == 1
+    assert L.mala_fwd(vp(), vp(), vp(), vp(), vp(), 1, 4, 2, 0, 128, 0, 0.1, 1.0, 0, None, 0,
+                      None, None) == 1
+    # null pointers and misaligned pointers
+    assert L.mala_fwd(None, vp(), vp(), vp(), vp(), 1, 4, 2, 128, 128, 0, 0.1, 1.0, 0, None, 0,
+                      None, None) == 1
+    assert L.mala_fwd(ctypes.c_void_p(16 * 1024 + 2), vp(), vp(), vp(), vp(), 1, 4, 2, 128, 128,
+                      0, 0.1, 1.0, 0, None, 0, None, None) == 1
+    # unsupported head dim for the bf16 tensor-core path
+    assert L.mala_fwd(vp(), vp(), vp(), vp(), vp(), 1, 4, 2, 128, 96, 0, 0.1, 1.0, 0, None, 0,
+                      None, None) == 2
+    # decode: split count out of range
+    assert L.mala_decode(vp(), vp(), vp(), vp(), vp(), 1, 4, 2, 256, 128, 0, 0.1, 1.0, 3, 0,
+                         None, 0, None, None) == 1
+    # backward: bad dtype code
+    assert L.mala_bwd(vp(), vp(), vp(), vp(), vp(), vp(), vp(), vp(), vp(), 1, 4, 2, 128, 128, 7,
+                      0.1, 1.0, 0, None, 0, None, None) == 1
+    # workspace too small (checked before any CUDA call)
+    assert L.mala_fwd(vp(), vp(), vp(), vp(), vp(), 1, 4, 2, 128, 128, 0, 0.1, 1.0, 0, vp(), 8,
+                      None, None) == 5
+
+
+def test_workspace_sizes_and_split_rule(lib):
+    B, H, Hkv, L, d = 1, 32, 8, 32768, 128
+    assert lib.fwd_workspace_bytes(B, H, Hkv, L, d) == 256
+    assert lib.bwd_workspace_bytes(B, H, Hkv, L, d) >= 256 + B * L * H * d * 4 + B * H * L * 4
+    S = lib.decode_num_splits(4, 32, 8, 131072)
+    assert 1 <= S <= 1024
+    assert lib.decode_num_splits(4, 32, 8, 131072) == S  # deterministic
+    assert lib.decode_workspace_bytes(4, 32, 8, 131072, 128, 0, S) >= 256 + 4 * 32 * S * 129 * 4
+    assert lib.decode_num_splits(1, 4, 1, 100) == 1
+    assert lib.decode_workspace_bytes(1, 4, 2, 256, 128, 0, 5) == 0  # 5 splits > 2 tiles
+
+
+def test_bench_accounting():
+    sys.path.insert(0, ROOT)
+    import bench
+    from mass_adaptive_sparse_fwd_b200 import synth
+
+    w = synth.WORKLOADS["sinkband32k"]
+    full = bench.fwd_bwd_flops(w, 1.0, 1.0)
+    # tile-granular dense counts exceed the exact causal counts only by the diagonal halves
+    assert 1.0 < full["fwd_exec"] / full["fwd_dense_eq"] < 1.01
+    assert 1.0 < full["bwd_exec"] / full["bwd_dense_eq"] < 1.01
+    none = bench.fwd_bwd_flops(w, 0.0, 0.0)
+    assert none["fwd_exec"] == pytest.approx(full["fwd_exec"] / 2)
+    assert none["bwd_exec"] == pytest.approx(full["bwd_exec"] / 5)
+    wd = synth.WORKLOADS["decode128k"]
+    kbytes = wd.B * wd.H_kv * wd.L * wd.d * 2
+    assert bench.decode_bytes(wd, 0, 1) > kbytes
+    assert bench.decode_bytes(wd, 10, 1) - bench.decode_bytes(wd, 0, 1) == 10 * 128 * 128 * 2
+
+
+_DIST_CHILD = r"""
+import os, sys
+sys.path.insert(0, {root!r})
+import bench
+d = bench.Dist().init("gloo")
+r = d.rank
+w = bench.rank_workload(bench.synth.WORKLOADS["sinkband32k"], r)
+v = d.max(10.0 + r)
+d.barrier()
+print(f"rank={{r}} seed={{w.seed}} max={{v}}", flush=True)
+d.close()
+"""
+
+
+def test_bench_two_ranks_gloo(tmp_path):
+    script = tmp_path / "child.py"
+    script.write_text(_DIST_CHILD.format(root=ROOT))
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node=2",
+           "--master-addr", "127.0.0.1", "--master-port", "29533", str(script)]
+    out = subprocess.run(cmd, capture_output=True, text=True, timeout=180)
+    assert out.returncode == 0, out.stderr[-2000:]
+    found = sorted(re.findall(r"rank=\d seed=\d+ max=[\d.]+", out.stdout))
+    assert found == ["rank=0 seed=3 max=11.0", "rank=1 seed=1003 max=11.0"], out.stdout
