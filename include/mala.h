@@ -106,6 +106,28 @@ mala_status mala_decode(const void* q, const void* Kc, const void* Vc, void* O, 
                         float tau, int num_splits, unsigned flags, void* workspace,
                         size_t workspace_bytes, uint8_t* tile_mask, void* stream);
 
+/*
+ * mala_decode_noalloc - mala_decode for callers that cannot allocate device memory.
+ * The attention page has no counterpart to this entry point; it exists for runtimes
+ * that forbid allocation on their hot path (a fixed memory plan after warm-up, a plugin
+ * inside a framework that owns the device allocator, code that must not call
+ * cudaMalloc or cudaMallocAsync per call).
+ *   Same arguments and results as mala_decode without the workspace: the scratch comes
+ *   from a fixed array of MALA_DECODE_NOALLOC_SCRATCH_BYTES compiled into the library,
+ *   which every GPU that loads the library holds until the process exits.  Calls whose
+ *   mala_decode_workspace_bytes() exceeds that size return MALA_ERR_WORKSPACE.
+ *   The first call on a device looks up the array's device address (once per device,
+ *   with that device current); make that first call before any stream capture.
+ *   All calls on a device share the array: calls whose work overlaps on the GPU (two
+ *   streams at once) race and must be serialised by the caller.  Device-side wait
+ *   timeouts are recorded in the internal array and are not reported by this call.
+ */
+#define MALA_DECODE_NOALLOC_SCRATCH_BYTES (4u << 20)
+mala_status mala_decode_noalloc(const void* q, const void* Kc, const void* Vc, void* O,
+                                float* LSE, int B, int H, int H_kv, int Nk, int d, int dtype,
+                                float scale, float tau, int num_splits, unsigned flags,
+                                uint8_t* tile_mask, void* stream);
+
 /* Workspace sizes (bytes) for the calls above; 0 on invalid arguments. */
 size_t mala_fwd_workspace_bytes(int B, int H, int H_kv, int L, int d, int dtype);
 size_t mala_bwd_workspace_bytes(int B, int H, int H_kv, int L, int d, int dtype);

@@ -24,7 +24,7 @@ MALA_BF16, MALA_FP32 = 0, 1
 MALA_FLAG_ALWAYS_TEST = 1
 TILE = 128
 
-EXPORTED = ("mala_fwd", "mala_bwd", "mala_decode", "mala_fwd_workspace_bytes",
+EXPORTED = ("mala_fwd", "mala_bwd", "mala_decode", "mala_decode_noalloc", "mala_fwd_workspace_bytes",
             "mala_bwd_workspace_bytes", "mala_decode_workspace_bytes", "mala_decode_num_splits",
             "mala_read_device_error", "mala_set_wait_budget_ns", "mala_status_string",
             "mala_version")
@@ -48,6 +48,9 @@ def load_library(path: str = _LIB_PATH) -> ctypes.CDLL:
                              cu, vp, sz, vp, vp]
     lib.mala_decode.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, cf, cf, ci, cu, vp, sz,
                                 vp, vp]
+    lib.mala_decode_noalloc.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, cf, cf, ci, cu,
+                                        vp, vp]
+    lib.mala_decode_noalloc.restype = ci
     for f in ("mala_fwd", "mala_bwd", "mala_decode", "mala_read_device_error",
               "mala_set_wait_budget_ns"):
         getattr(lib, f).restype = ci
@@ -168,6 +171,23 @@ def mala_decode(q, Kc, Vc, scale, tau, num_splits=0, O=None, LSE=None, flags=0, 
                           _dtype_code(q), float(scale), float(tau), int(num_splits), flags,
                           _ptr(workspace), ws_bytes, _ptr(tile_mask), _stream(stream))
     _check("mala_decode", st)
+    return O, LSE
+
+
+def mala_decode_noalloc(q, Kc, Vc, scale, tau, num_splits=0, O=None, LSE=None, flags=0,
+                        tile_mask=None, stream=None):
+    """Split-KV decode that allocates nothing on the device: its scratch is a fixed
+    array inside the library (for callers that may not allocate device memory on their
+    hot path).  Calls on one device share that array, so they must not overlap on the
+    GPU.  Returns (O [B,H,d], LSE [B,H])."""
+    B, H, d = q.shape
+    Nk, H_kv = Kc.shape[1], Kc.shape[2]
+    O = torch.empty_like(q) if O is None else O
+    LSE = torch.empty((B, H), dtype=torch.float32, device=q.device) if LSE is None else LSE
+    st = _lib.mala_decode_noalloc(_ptr(q), _ptr(Kc), _ptr(Vc), _ptr(O), _ptr(LSE), B, H, H_kv,
+                                  Nk, d, _dtype_code(q), float(scale), float(tau),
+                                  int(num_splits), flags, _ptr(tile_mask), _stream(stream))
+    _check("mala_decode_noalloc", st)
     return O, LSE
 
 
