@@ -374,9 +374,16 @@ def run_mala(args, dist: Dist):
     traffic = None
     prof = os.path.join(ROOT, "profiles", "roofline_traffic.json")
     if os.path.exists(prof):
+        import hashlib
+
         with open(prof) as f:
             tr = json.load(f)
-        traffic = tr.get("mala_bwd_kernel_bytes_per_launch")
+        src = os.path.join(ROOT, "mass_adaptive_sparse_fwd_b200", "csrc", "mala_bwd.cu")
+        with open(src, "rb") as f:
+            sha = hashlib.sha256(f.read()).hexdigest()[:16]
+        # counters only count for the kernel source they were taken on
+        if tr.get("source_sha256_16") == sha:
+            traffic = tr.get("mala_bwd_kernel_bytes_per_launch")
 
     # end to end through the C ABI with host buffers (pinned), copies in the timed region
     e2e = None
