@@ -121,3 +121,14 @@ def test_bwd_sinkband32k_sampled(orc, mala):
     T = w.L // 128
     check_bwd(orc, mala, w, synth.make_training(w), 1.0,
               kv_units=[(0, 7, T - 1), (0, 3, T // 2)], q_units=[(0, 31, T - 1), (0, 0, 5)])
+
+
+@pytest.mark.parametrize("tau", [0.0, 1.0])
+def test_bwd_tiny256_fp32(orc, mala, tau):
+    w = synth.WORKLOADS["tiny256"]
+    check_bwd(orc, mala, w, synth.make_training(w), tau)
+
+
+def test_bwd_fp32_ragged_gqa(orc, mala):
+    w, inp = synth.small_training(B=2, H=4, Hkv=2, L=200, d=32, dtype="fp32", structure="peaked")
+    check_bwd(orc, mala, w, inp, 1.0)

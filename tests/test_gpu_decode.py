@@ -87,3 +87,10 @@ def test_decode128k_full(orc, mala):
     # splits that hold a planted key skip the tiles after it; splits without one test
     # against a small diffuse normaliser and keep most tiles (the oracle agrees)
     assert (mask == 0).any()
+
+
+@pytest.mark.parametrize("tau", [0.0, 1.0])
+def test_decode_fp32(orc, mala, tau):
+    w = synth.Workload("fp32_decode", 2, 4, 2, 700, 64, "fp32", "planted", 23, decode=True)
+    inp = synth.make_decode(w)
+    check_decode(orc, mala, inp, w.scale, tau, 2, dtype="fp32")

@@ -102,3 +102,14 @@ def test_fwd_sinkband32k_sampled(orc, mala):
     inp = synth.make_training(w)
     T = w.L // 128
     check_fwd(orc, mala, w, inp, 1.0, units=_units(w.B, w.H, T, 4, seed=5))
+
+
+@pytest.mark.parametrize("tau", [0.0, 1.0])
+def test_fwd_tiny256_fp32(orc, mala, tau):
+    w = synth.WORKLOADS["tiny256"]
+    check_fwd(orc, mala, w, synth.make_training(w), tau)
+
+
+def test_fwd_fp32_ragged_gqa(orc, mala):
+    w, inp = synth.small_training(B=2, H=4, Hkv=2, L=200, d=32, dtype="fp32", structure="peaked")
+    check_fwd(orc, mala, w, inp, 1.0)
