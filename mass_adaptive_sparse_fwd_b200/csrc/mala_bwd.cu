@@ -20,15 +20,19 @@
 //   dV += P^T dO_i,  dK += dS^T Q_i,  dQ_i += dS K_j  (fp32 reduction into global).
 //
 // Warp roles (512 threads):
-//   warp 0       TMA producer: K_j and V_j once per unit; Q_i and dO_i per tile
-//                (dO is fetched with Q, ahead of the decision, like V in the forward).
+//   warp 0       TMA producer: K_j and V_j once per unit; Q_i (2-stage ring) and dO_i
+//                (1 stage) per tile.  dO is fetched ahead of the decision, like V in the
+//                forward.
 //   warp 1       TMEM owner and UMMA issuer.
 //   warps 4-11   two softmax warpgroups: thread = key row (TMEM lane); warpgroup w
 //                owns query columns [64 w, 64 w + 64).  They evaluate the test (one
 //                bar.red.or over both groups), write P^T into TMEM and dS^T into shared
 //                memory.
-//   warps 12-15  dQ drain (TMEM -> red.global.add.v4.f32) and the per-unit dK / dV
-//                epilogue.
+//   warps 12-15  dQ drain and the per-unit dK / dV epilogue.  The dQ tile is copied
+//                from TMEM into a 128-byte-swizzled fp32 staging buffer (64 columns at a
+//                time) and added into the global fp32 accumulator with TMA bulk
+//                reductions (cp.reduce.async.bulk.tensor .add); its TMEM columns are
+//                released as soon as they have been read.
 // TMEM columns: S^T [0,128) (P^T bf16 overwrites [0,64)), dP^T [128,256) (the dQ tile
 // of the same step overwrites it once dS^T has been formed), dV [256, 256+D),
 // dK [256+D, 256+2D).
@@ -56,9 +60,11 @@ template <int D>
 struct BwdCfg {
   static constexpr int TILE_BYTES = kTile * D * 2;
   static constexpr int BOXES = D / 64;
-  static constexpr int NQ = 2;  // Q / dO ring stages
-  // K, V, NQ x (Q, dO), dS^T (128 x 128 bf16)
-  static constexpr int SMEM = 2 * TILE_BYTES + 2 * NQ * TILE_BYTES + kTile * kTile * 2;
+  static constexpr int NQ = 2;  // Q ring stages (dO has one)
+  static constexpr int STAGE_BYTES = 2 * 16384;  // dQ staging: two [128 x 32] fp32 boxes
+  // K, V, NQ x Q, dO, dS^T (128 x 128 bf16), dQ staging
+  static constexpr int SMEM =
+      2 * TILE_BYTES + NQ * TILE_BYTES + TILE_BYTES + kTile * kTile * 2 + STAGE_BYTES;
 };
 
 struct BwdParams {
@@ -78,6 +84,7 @@ struct BwdParams {
 struct BwdShared {
   uint64_t kv_full, kv_empty;
   uint64_t q_full[2], q_empty[2];
+  uint64_t do_full, do_empty;
   uint64_t s_full, p_full, dp_full, ds_full, dq_full, dq_empty, acc_full, acc_empty;
   uint64_t sched_full[2], sched_empty[2];
   uint64_t final_bar;
@@ -115,29 +122,20 @@ __device__ __forceinline__ void tile_hi(const BwdParams& p, const BUnit& w, int 
   i = w.j + n % per;
 }
 
-__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
-  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b),
-               "f"(c), "f"(d)
-               : "memory");
-}
-
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
 template <int D, bool kScreen>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     mala_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
-                    const BwdParams p) {
+                    const __grid_constant__ CUtensorMap tmdQ, const BwdParams p) {
   using C = BwdCfg<D>;
   constexpr int NQ = C::NQ;
   extern __shared__ __align__(1024) uint8_t smem[];
   uint8_t* sK = smem;
   uint8_t* sV = sK + C::TILE_BYTES;
   uint8_t* sQ = sV + C::TILE_BYTES;                 // NQ tiles
-  uint8_t* sdO = sQ + NQ * C::TILE_BYTES;           // NQ tiles
-  uint8_t* sdS = sdO + NQ * C::TILE_BYTES;          // 128 x 128 bf16, two 64-column atoms
+  uint8_t* sdO = sQ + NQ * C::TILE_BYTES;           // 1 tile
+  uint8_t* sdS = sdO + C::TILE_BYTES;               // 128 x 128 bf16, two 64-column atoms
+  uint8_t* sdQ = sdS + kTile * kTile * 2;           // dQ staging, two [128 x 32] fp32 boxes
   __shared__ BwdShared sh;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -153,6 +151,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_init(&sh.q_full[s], 1);
       mbar_init(&sh.q_empty[s], 1);
     }
+    mbar_init(&sh.do_full, 1);
+    mbar_init(&sh.do_empty, 1);
     mbar_init(&sh.s_full, 1);
     mbar_init(&sh.p_full, 256);
     mbar_init(&sh.dp_full, 1);
@@ -187,7 +187,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
       tma_prefetch_desc(&tmdO);
-      uint32_t c = 0, nu = 0;
+      tma_prefetch_desc(&tmdQ);
+      uint32_t c = 0, nu = 0, ndo = 0;
       bool ok = true;
       for (uint32_t k = 0; ok; ++k) {
         const int ring = k & 1;
@@ -209,13 +210,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           tile_hi(p, w, n, h, i);
           const int st = c % NQ;
           if (c >= NQ && !(ok = mbar_wait(&sh.q_empty[st], ((c / NQ) - 1) & 1, ast, 3))) break;
-          mbar_arrive_expect_tx(&sh.q_full[st], 2 * C::TILE_BYTES);
-          for (int x = 0; x < C::BOXES; ++x) {
+          mbar_arrive_expect_tx(&sh.q_full[st], C::TILE_BYTES);
+          for (int x = 0; x < C::BOXES; ++x)
             tma_load_4d(sQ + st * C::TILE_BYTES + x * 16384, &tmQ, &sh.q_full[st], x * 64, h,
                         i * kTile, w.b);
-            tma_load_4d(sdO + st * C::TILE_BYTES + x * 16384, &tmdO, &sh.q_full[st], x * 64, h,
-                        i * kTile, w.b);
-          }
+          // dO has a single stage: released by the MMA once dP^T and dV of tile c-1 are done
+          if (c >= 1 && !(ok = mbar_wait(&sh.do_empty, (c - 1) & 1, ast, 5))) break;
+          mbar_arrive_expect_tx(&sh.do_full, C::TILE_BYTES);
+          for (int x = 0; x < C::BOXES; ++x)
+            tma_load_4d(sdO + x * 16384, &tmdO, &sh.do_full, x * 64, h, i * kTile, w.b);
+          ndo = c + 1;
         }
       }
       if (!ok) {
@@ -226,6 +230,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         if (nu > 0) mbar_wait(&sh.kv_full, (nu - 1) & 1, drain, 4);
         for (uint32_t cc = (c > NQ ? c - NQ : 0); cc < c; ++cc)
           mbar_wait(&sh.q_full[cc % NQ], (cc / NQ) & 1, drain, 4);
+        if (ndo > 0) mbar_wait(&sh.do_full, (ndo - 1) & 1, drain, 4);
       }
     }
   } else if (warp == 1) {
@@ -265,10 +270,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         for (int n = 0; n < w.ntiles && ok; ++n, ++c, ++ntile) {
           const int st = c % NQ;
           const uint32_t aQ = smem_u32(sQ + st * C::TILE_BYTES);
-          const uint32_t adO = smem_u32(sdO + st * C::TILE_BYTES);
+          const uint32_t adO = smem_u32(sdO);
           if (!(ok = mbar_wait(&sh.p_full, ntile & 1, ast, 13))) break;
           tc_fence_after();
           const bool keep = sh.dec != 0;
+          // dO(c) is loaded for every tile; its stage is released after dP^T / dV
+          if (!(ok = mbar_wait(&sh.do_full, c & 1, ast, 20))) break;
           if (keep) {
             // dP^T reuses the columns of the previous dQ tile: wait for its drain
             if (ntile > 0 && !(ok = mbar_wait(&sh.dq_empty, (ntile - 1) & 1, ast, 14))) break;
@@ -289,6 +296,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
               umma_ts(tdV, tS + kk * 8, sdesc_sw128(adO + kk * 2048, 16384, 1024), id_acc,
                       (acc_started || kk > 0) ? 1u : 0u);
           }
+          umma_commit(&sh.do_empty);
           // next tile's S^T (after dV has consumed P^T from the same columns)
           if (n + 1 < w.ntiles) {
             const uint32_t c1 = c + 1;
@@ -356,29 +364,37 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const BUnit w = decode_bunit(p, u);
       const int krow = w.j * kTile + r;
       const bool kvalid = krow < p.L;
+      // per-column constants (LSE in log2 units, threshold, D) of tile n, loaded one tile
+      // ahead into registers by threads tw < 64 and published through shared memory
+      auto load_cols = [&](int n, float& l2, float& c2, float& ds) {
+        int h, i;
+        tile_hi(p, w, n, h, i);
+        const int q = i * kTile + wg * 64 + tw;
+        c2 = INFINITY; l2 = 0.f; ds = 0.f;
+        if (tw < 64 && q < p.L) {
+          const size_t idx = (static_cast<size_t>(w.b) * p.H + h) * p.L + q;
+          l2 = p.LSE[idx] * kLog2e;
+          ds = p.Dsum[idx];
+          c2 = kScreen ? l2 + (p.log2_tau - __log2f(static_cast<float>(q + 1))) : NEG_INF;
+        }
+      };
+      float nl2, nc2, nds;
+      load_cols(0, nl2, nc2, nds);
       for (int n = 0; n < w.ntiles; ++n, ++ntile) {
         int h, i;
         tile_hi(p, w, n, h, i);
-        // per-column constants of this tile (warpgroup-private buffers)
         named_bar_sync(2 + wg, 128);  // previous tile's readers are done
         if (tw < 64) {
-          const int q = i * kTile + wg * 64 + tw;
-          float c2 = INFINITY, l2 = 0.f, ds = 0.f;
-          if (q < p.L) {
-            const size_t idx = (static_cast<size_t>(w.b) * p.H + h) * p.L + q;
-            l2 = p.LSE[idx] * kLog2e;
-            ds = p.Dsum[idx];
-            c2 = kScreen ? l2 + (p.log2_tau - __log2f(static_cast<float>(q + 1))) : NEG_INF;
-          }
-          sh.c2[wg][tw] = c2;
-          sh.lse2[wg][tw] = l2;
-          sh.dsum[wg][tw] = ds;
+          sh.c2[wg][tw] = nc2;
+          sh.lse2[wg][tw] = nl2;
+          sh.dsum[wg][tw] = nds;
         }
         named_bar_sync(2 + wg, 128);
-        const bool got = mbar_wait(&sh.s_full, ntile & 1, ast, 21);
+        if (n + 1 < w.ntiles) load_cols(n + 1, nl2, nc2, nds);
+        const bool got = mbar_wait_warp(&sh.s_full, ntile & 1, ast, 21);
         tc_fence_after();
         uint32_t v[2][32];
-        if (__all_sync(0xffffffffu, got)) {
+        if (got) {
           tmem_ld32(tS + lane_off + wg * 64, v[0]);
           tmem_ld32(tS + lane_off + wg * 64 + 32, v[1]);
           tmem_wait_ld();
@@ -435,13 +451,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tc_fence_before();
         mbar_arrive(&sh.p_full);
         // dS^T = P^T o (dP^T - D) * scale -> bf16, swizzled K-major rows in shared memory
-        const bool dp_ok = mbar_wait(&sh.dp_full, nret & 1, ast, 22);
+        const bool dp_ok = mbar_wait_warp(&sh.dp_full, nret & 1, ast, 22);
         ++nret;
         // the dS^T buffer is free once the previous tile's dK / dQ MMAs completed
         bool buf_ok = true;
-        if (ntile > 0) buf_ok = mbar_wait(&sh.dq_full, (ntile - 1) & 1, ast, 23);
+        if (ntile > 0) buf_ok = mbar_wait_warp(&sh.dq_full, (ntile - 1) & 1, ast, 23);
         tc_fence_after();
-        if (__all_sync(0xffffffffu, dp_ok && buf_ok)) {
+        if (dp_ok && buf_ok) {
 #pragma unroll
           for (int a = 0; a < 2; ++a) {
             uint32_t dp[32];
@@ -486,30 +502,51 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       for (int n = 0; n < w.ntiles; ++n, ++ntile) {
         int h, i;
         tile_hi(p, w, n, h, i);
-        const bool got_dq = __all_sync(0xffffffffu, mbar_wait(&sh.dq_full, ntile & 1, ast, 31));
+        const bool got_dq = mbar_wait_warp(&sh.dq_full, ntile & 1, ast, 31);
         tc_fence_after();
-        if (got_dq && sh.dq_flag[ntile & 1]) {
-          const int q = i * kTile + r;
-          float* dst = p.dQacc + ((static_cast<size_t>(w.b) * p.L + q) * p.H + h) * D;
+        // the drain below holds named barriers: decide it uniformly for the 128 threads
+        const bool drain = named_bar_or(5, 128, got_dq && sh.dq_flag[ntile & 1] != 0);
+        if (!drain) {
+          tc_fence_before();
+          mbar_arrive(&sh.dq_empty);
+          continue;
+        }
+        // dQ tile (row r of query block i): 64 columns per round through the staging
+        // buffer, TMA bulk add into the fp32 accumulator.  The TMEM columns are released
+        // right after the last round has been loaded into registers.
 #pragma unroll
-          for (int a = 0; a < D / 32; ++a) {
-            uint32_t o[32];
-            tmem_ld32(tdP + lane_off + a * 32, o);
-            tmem_wait_ld();
-            if (q < p.L) {
+        for (int half = 0; half < D / 64; ++half) {
+          uint32_t o[2][32];
+          tmem_ld32(tdP + lane_off + half * 64, o[0]);
+          tmem_ld32(tdP + lane_off + half * 64 + 32, o[1]);
+          tmem_wait_ld();
+          if (half == D / 64 - 1) {
+            tc_fence_before();
+            mbar_arrive(&sh.dq_empty);
+          }
+          // staging buffer free: the previous round's bulk reads have completed
+          if (tid == 384) bulk_wait_read_all();
+          named_bar_sync(5, 128);
 #pragma unroll
-              for (int e = 0; e < 8; ++e)
-                red_add_v4(dst + a * 32 + 4 * e, __uint_as_float(o[4 * e]),
-                           __uint_as_float(o[4 * e + 1]), __uint_as_float(o[4 * e + 2]),
-                           __uint_as_float(o[4 * e + 3]));
-            }
+          for (int box = 0; box < 2; ++box)
+#pragma unroll
+            for (int ch = 0; ch < 8; ++ch)
+              *reinterpret_cast<uint4*>(sdQ + box * 16384 + sw128_offset(r, ch)) =
+                  make_uint4(o[box][4 * ch], o[box][4 * ch + 1], o[box][4 * ch + 2],
+                             o[box][4 * ch + 3]);
+          fence_proxy_async_smem();
+          named_bar_sync(5, 128);
+          if (tid == 384) {
+#pragma unroll
+            for (int box = 0; box < 2; ++box)
+              tma_reduce_add_4d(&tmdQ, sdQ + box * 16384, half * 64 + box * 32, h, i * kTile,
+                                w.b);
+            bulk_commit_group();
           }
         }
-        tc_fence_before();
-        mbar_arrive(&sh.dq_empty);
       }
       // unit epilogue: dK, dV of key block j
-      const bool got_acc = __all_sync(0xffffffffu, mbar_wait(&sh.acc_full, nu & 1, ast, 32));
+      const bool got_acc = mbar_wait_warp(&sh.acc_full, nu & 1, ast, 32);
       tc_fence_after();
       const bool valid_acc = sh.acc_valid != 0;
       const int krow = w.j * kTile + r;
@@ -547,6 +584,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_arrive(&sh.acc_empty);
       ++nu;
     }
+    // every dQ reduction of this CTA must have landed before the kernel ends
+    if (tid == 384) bulk_wait_all();
   }
 
   tc_fence_before();
@@ -617,13 +656,38 @@ mala_status fp32_bwd(const float* Q, const float* K, const float* V, const float
 template <int D, bool kScreen>
 static cudaError_t launch_bwd_main(const CUtensorMap& tq, const CUtensorMap& tk,
                                    const CUtensorMap& tv, const CUtensorMap& tdo,
-                                   const BwdParams& p, int grid, cudaStream_t stream) {
+                                   const CUtensorMap& tdq, const BwdParams& p, int grid,
+                                   cudaStream_t stream) {
   auto kern = mala_bwd_kernel<D, kScreen>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        BwdCfg<D>::SMEM);
   if (e != cudaSuccess) return e;
-  kern<<<grid, kBwdThreads, BwdCfg<D>::SMEM, stream>>>(tq, tk, tv, tdo, p);
+  kern<<<grid, kBwdThreads, BwdCfg<D>::SMEM, stream>>>(tq, tk, tv, tdo, tdq, p);
   return cudaGetLastError();
+}
+
+// fp32 [n3][n2][n1][n0] tensor, box {32, 1, 128, 1} (128-byte rows), 128-byte swizzle.
+static bool make_f32_reduce_map(CUtensorMap* m, void* base, int n0, int n1, int n2, int n3) {
+  typedef CUresult (*EncodeFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                               const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                               const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                               CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+  void* f = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) !=
+          cudaSuccess ||
+      q != cudaDriverEntryPointSuccess)
+    return false;
+  cuuint64_t dims[4] = {(cuuint64_t)n0, (cuuint64_t)n1, (cuuint64_t)n2, (cuuint64_t)n3};
+  cuuint64_t strides[3] = {(cuuint64_t)n0 * 4, (cuuint64_t)n0 * n1 * 4,
+                           (cuuint64_t)n0 * n1 * n2 * 4};
+  cuuint32_t box[4] = {32, 1, 128, 1};
+  cuuint32_t es[4] = {1, 1, 1, 1};
+  return reinterpret_cast<EncodeFn>(f)(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, base, dims, strides,
+                                       box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                                       CU_TENSOR_MAP_SWIZZLE_128B,
+                                       CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                                       CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 mala_status bwd_dispatch(const void* Q, const void* K, const void* V, const void* O,
@@ -647,6 +711,8 @@ mala_status bwd_dispatch(const void* Q, const void* K, const void* V, const void
   const size_t acc_bytes = static_cast<size_t>(B) * L * H * d * sizeof(float);
   float* dQacc = reinterpret_cast<float*>(ws + kWorkspaceHeader);
   float* Dsum = reinterpret_cast<float*>(ws + kWorkspaceHeader + ((acc_bytes + 255) / 256) * 256);
+  CUtensorMap tdq;
+  if (!make_f32_reduce_map(&tdq, dQacc, d, H, L, B)) return MALA_ERR_CUDA;
   if (cudaMemsetAsync(hdr + kHdrSched0, 0, 3 * sizeof(uint32_t), stream) != cudaSuccess)
     return MALA_ERR_CUDA;
   const long long rows = static_cast<long long>(B) * L * H;
@@ -676,11 +742,11 @@ mala_status bwd_dispatch(const void* Q, const void* K, const void* V, const void
   const int grid = p.n_units < sm_count() ? p.n_units : sm_count();
   cudaError_t e;
   if (d == 128)
-    e = screen ? launch_bwd_main<128, true>(tq, tk, tv, tdo, p, grid, stream)
-               : launch_bwd_main<128, false>(tq, tk, tv, tdo, p, grid, stream);
+    e = screen ? launch_bwd_main<128, true>(tq, tk, tv, tdo, tdq, p, grid, stream)
+               : launch_bwd_main<128, false>(tq, tk, tv, tdo, tdq, p, grid, stream);
   else
-    e = screen ? launch_bwd_main<64, true>(tq, tk, tv, tdo, p, grid, stream)
-               : launch_bwd_main<64, false>(tq, tk, tv, tdo, p, grid, stream);
+    e = screen ? launch_bwd_main<64, true>(tq, tk, tv, tdo, tdq, p, grid, stream)
+               : launch_bwd_main<64, false>(tq, tk, tv, tdo, tdq, p, grid, stream);
   if (e != cudaSuccess) return MALA_ERR_CUDA;
   const long long n4 = rows * d / 4;
   mala_bwd_dq<<<static_cast<unsigned>((n4 + 255) / 256), 256, 0, stream>>>(
