@@ -16,8 +16,9 @@
 // always recomputed.  The offline test of Eq. (4): the tile is retained iff some legal
 // entry has s_kq * scale - LSE_q >= log(tau / L_q) (L_q = q + 1), evaluated in log2
 // units.  Only a retained tile runs the post-score work:
-//   P^T = exp(S^T - LSE),  dP^T = V_j dO_i^T,  dS^T = P^T o (dP^T - D) * scale,
-//   dV += P^T dO_i,  dK += dS^T Q_i,  dQ_i += dS K_j  (fp32 reduction into global).
+//   P^T = exp(S^T - LSE),  dP^T = V_j dO_i^T,  dS^T = P^T o (dP^T - D),
+//   dV += P^T dO_i,  dK += scale dS^T Q_i,  dQ_i += scale dS K_j  (fp32 reduction into
+//   global; the scale is applied when dK is stored and when dQ is converted).
 //
 // Warp roles (512 threads):
 //   warp 0       TMA producer: K_j and V_j once per unit; Q_i (2-stage ring) and dO_i
@@ -88,9 +89,11 @@ struct BwdShared {
   uint64_t s_full, p_full, dp_full, ds_full, dq_full, dq_empty, acc_full, acc_empty;
   uint64_t sched_full[2], sched_empty[2];
   uint64_t final_bar;
-  float c2[2][64];   // per softmax warpgroup: LSE2_q + log2(tau / L_q) (+inf if q >= L)
-  float lse2[2][64]; // LSE_q * log2(e)
-  float dsum[2][64]; // D_q
+  // per softmax warpgroup and query column: LSE_q in log2 units (+inf past L, so the
+  // probability is 0 there), the threshold log2(tau / L_q) and D_q
+  alignas(16) float lse2[2][64];
+  alignas(16) float thr2[2][64];
+  alignas(16) float dsum[2][64];
   int sched_ring[2];
   uint32_t dec;      // decision of the current tile (1 = retained)
   uint32_t dq_flag[2];
@@ -366,31 +369,31 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const bool kvalid = krow < p.L;
       // per-column constants (LSE in log2 units, threshold, D) of tile n, loaded one tile
       // ahead into registers by threads tw < 64 and published through shared memory
-      auto load_cols = [&](int n, float& l2, float& c2, float& ds) {
+      auto load_cols = [&](int n, float& l2, float& t2, float& ds) {
         int h, i;
         tile_hi(p, w, n, h, i);
         const int q = i * kTile + wg * 64 + tw;
-        c2 = INFINITY; l2 = 0.f; ds = 0.f;
+        l2 = INFINITY; t2 = INFINITY; ds = 0.f;
         if (tw < 64 && q < p.L) {
           const size_t idx = (static_cast<size_t>(w.b) * p.H + h) * p.L + q;
           l2 = p.LSE[idx] * kLog2e;
           ds = p.Dsum[idx];
-          c2 = kScreen ? l2 + (p.log2_tau - __log2f(static_cast<float>(q + 1))) : NEG_INF;
+          t2 = kScreen ? p.log2_tau - __log2f(static_cast<float>(q + 1)) : NEG_INF;
         }
       };
-      float nl2, nc2, nds;
-      load_cols(0, nl2, nc2, nds);
+      float nl2, nt2, nds;
+      load_cols(0, nl2, nt2, nds);
       for (int n = 0; n < w.ntiles; ++n, ++ntile) {
         int h, i;
         tile_hi(p, w, n, h, i);
         named_bar_sync(2 + wg, 128);  // previous tile's readers are done
         if (tw < 64) {
-          sh.c2[wg][tw] = nc2;
           sh.lse2[wg][tw] = nl2;
+          sh.thr2[wg][tw] = nt2;
           sh.dsum[wg][tw] = nds;
         }
         named_bar_sync(2 + wg, 128);
-        if (n + 1 < w.ntiles) load_cols(n + 1, nl2, nc2, nds);
+        if (n + 1 < w.ntiles) load_cols(n + 1, nl2, nt2, nds);
         const bool got = mbar_wait_warp(&sh.s_full, ntile & 1, ast, 21);
         tc_fence_after();
         uint32_t v[2][32];
@@ -404,19 +407,30 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
             for (int e = 0; e < 32; ++e) v[a][e] = 0xff800000u;
         }
-        // legal entries: key row valid, query q < L, and q >= k on the diagonal block
-        const int qlo = (i == w.j) ? (r - wg * 64) : -1;  // local column must be >= qlo
+        // a = log2 P = s * scale * log2(e) - LSE2_q (-inf past L through LSE2 = +inf);
+        // the tile is kept if some legal entry has a >= log2(tau / L_q) (Eq. 4).
+        // Causal masking is needed only on the diagonal block and past the last key.
+        // local column must be >= qlo: -1 off the diagonal, 64 for key rows past the end
+        const int qlo = !kvalid ? 64 : (i == w.j ? r - wg * 64 : -1);
         float ymax = NEG_INF;
+        const float4* l4 = reinterpret_cast<const float4*>(sh.lse2[wg]);
+        const float4* t4 = reinterpret_cast<const float4*>(sh.thr2[wg]);
 #pragma unroll
         for (int a = 0; a < 2; ++a)
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const int cl = a * 32 + e;
-            float x = __uint_as_float(v[a][e]) * p.scale_log2;
-            const bool legal = kvalid && cl >= qlo && sh.c2[wg][cl] != INFINITY;
-            x = legal ? x : NEG_INF;
-            v[a][e] = __float_as_uint(x);
-            if (kScreen) ymax = fmaxf(ymax, x - sh.c2[wg][cl]);
+          for (int e4 = 0; e4 < 8; ++e4) {
+            const float4 lv = l4[a * 8 + e4];
+            const float4 tv = t4[a * 8 + e4];
+            const float lq[4] = {lv.x, lv.y, lv.z, lv.w};
+            const float tq[4] = {tv.x, tv.y, tv.z, tv.w};
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              const int cl = a * 32 + e4 * 4 + c;
+              float x = fmaf(__uint_as_float(v[a][e4 * 4 + c]), p.scale_log2, -lq[c]);
+              x = (cl >= qlo) ? x : NEG_INF;
+              v[a][e4 * 4 + c] = __float_as_uint(x);
+              if (kScreen) ymax = fmaxf(ymax, x - tq[c]);
+            }
           }
         bool keep = true;
         if (kScreen) keep = named_bar_or(1, 256, ymax >= 0.f);
@@ -430,7 +444,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           mbar_arrive(&sh.p_full);
           continue;
         }
-        // P^T = exp2(x - LSE2) -> bf16 pairs into TMEM columns [32 wg, 32 wg + 32)
+        // P^T = exp2(a) -> bf16 pairs into TMEM columns [32 wg, 32 wg + 32)
         float pf[64];
 #pragma unroll
         for (int a = 0; a < 2; ++a) {
@@ -438,8 +452,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
             const int c0 = a * 32 + 2 * e;
-            const float p0 = fast_exp2(__uint_as_float(v[a][2 * e]) - sh.lse2[wg][c0]);
-            const float p1 = fast_exp2(__uint_as_float(v[a][2 * e + 1]) - sh.lse2[wg][c0 + 1]);
+            const float p0 = fast_exp2(__uint_as_float(v[a][2 * e]));
+            const float p1 = fast_exp2(__uint_as_float(v[a][2 * e + 1]));
             pf[c0] = p0;
             pf[c0 + 1] = p1;
             pk[e] = pack_bf16(p0, p1);
@@ -450,7 +464,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         if (tid == 128) sh.dec = 1;
         tc_fence_before();
         mbar_arrive(&sh.p_full);
-        // dS^T = P^T o (dP^T - D) * scale -> bf16, swizzled K-major rows in shared memory
+        // dS^T = P^T o (dP^T - D) -> bf16, swizzled K-major rows in shared memory (the
+        // softmax scale is applied to dK in the epilogue and to dQ in the final convert)
         const bool dp_ok = mbar_wait_warp(&sh.dp_full, nret & 1, ast, 22);
         ++nret;
         // the dS^T buffer is free once the previous tile's dK / dQ MMAs completed
@@ -463,16 +478,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             uint32_t dp[32];
             tmem_ld32(tdP + lane_off + wg * 64 + a * 32, dp);
             tmem_wait_ld();
+            const float4* d4 = reinterpret_cast<const float4*>(sh.dsum[wg]);
 #pragma unroll
             for (int ch = 0; ch < 4; ++ch) {  // 4 chunks of 8 columns = 16 bytes
+              const float4 da = d4[a * 8 + ch * 2], db = d4[a * 8 + ch * 2 + 1];
+              const float dq[8] = {da.x, da.y, da.z, da.w, db.x, db.y, db.z, db.w};
               uint32_t pk[4];
 #pragma unroll
               for (int e = 0; e < 4; ++e) {
                 const int c0 = a * 32 + ch * 8 + 2 * e;
-                const float d0 = pf[c0] * (__uint_as_float(dp[ch * 8 + 2 * e]) - sh.dsum[wg][c0]);
-                const float d1 =
-                    pf[c0 + 1] * (__uint_as_float(dp[ch * 8 + 2 * e + 1]) - sh.dsum[wg][c0 + 1]);
-                pk[e] = pack_bf16(d0 * p.scale, d1 * p.scale);
+                const float d0 = pf[c0] * (__uint_as_float(dp[ch * 8 + 2 * e]) - dq[2 * e]);
+                const float d1 = pf[c0 + 1] * (__uint_as_float(dp[ch * 8 + 2 * e + 1]) - dq[2 * e + 1]);
+                pk[e] = pack_bf16(d0, d1);
               }
               *reinterpret_cast<uint4*>(dsrow_base + sw128_offset(r, a * 4 + ch)) =
                   make_uint4(pk[0], pk[1], pk[2], pk[3]);
@@ -567,11 +584,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             for (int e8 = 0; e8 < 4; ++e8) {
               uint4 pk;
               const float* f = reinterpret_cast<const float*>(o) + e8 * 8;
+              const float sc = (which == 1) ? p.scale : 1.f;  // dK = scale * dS^T Q
               if (valid_acc) {
-                pk.x = pack_bf16(f[0], f[1]);
-                pk.y = pack_bf16(f[2], f[3]);
-                pk.z = pack_bf16(f[4], f[5]);
-                pk.w = pack_bf16(f[6], f[7]);
+                pk.x = pack_bf16(f[0] * sc, f[1] * sc);
+                pk.y = pack_bf16(f[2] * sc, f[3] * sc);
+                pk.z = pack_bf16(f[4] * sc, f[5] * sc);
+                pk.w = pack_bf16(f[6] * sc, f[7] * sc);
               } else {
                 pk = make_uint4(0u, 0u, 0u, 0u);
               }
@@ -628,14 +646,16 @@ __global__ void __launch_bounds__(256) mala_bwd_prep(const __nv_bfloat16* __rest
   }
 }
 
+// dQ = bf16(scale * accumulator): the accumulator holds dS K without the softmax scale.
 __global__ void __launch_bounds__(256) mala_bwd_dq(const float* __restrict__ acc,
-                                                   __nv_bfloat16* __restrict__ dQ, long long n4) {
+                                                   __nv_bfloat16* __restrict__ dQ, long long n4,
+                                                   float scale) {
   const long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (i >= n4) return;
   const float4 v = reinterpret_cast<const float4*>(acc)[i];
   uint2 pk;
-  pk.x = pack_bf16(v.x, v.y);
-  pk.y = pack_bf16(v.z, v.w);
+  pk.x = pack_bf16(v.x * scale, v.y * scale);
+  pk.y = pack_bf16(v.z * scale, v.w * scale);
   reinterpret_cast<uint2*>(dQ)[i] = pk;
 }
 
@@ -750,7 +770,7 @@ mala_status bwd_dispatch(const void* Q, const void* K, const void* V, const void
   if (e != cudaSuccess) return MALA_ERR_CUDA;
   const long long n4 = rows * d / 4;
   mala_bwd_dq<<<static_cast<unsigned>((n4 + 255) / 256), 256, 0, stream>>>(
-      dQacc, static_cast<__nv_bfloat16*>(dQ), n4);
+      dQacc, static_cast<__nv_bfloat16*>(dQ), n4, scale);
   return cudaGetLastError() == cudaSuccess ? MALA_OK : MALA_ERR_CUDA;
 }
 

@@ -315,39 +315,37 @@ __global__ void __launch_bounds__(384, 1)
         const bool got = mbar_wait(&sh.s_full[s], ns & 1, ast, 21);
         ++ns;
         tc_fence_after();
-        uint32_t v[4][32];
-        if (__all_sync(0xffffffffu, got)) {
+        // pass 1: row maximum of the raw scores (the scale is positive, so it commutes
+        // with max), 64 columns at a time; only the diagonal tile and rows past the end
+        // need masking (keys c <= r are legal on the diagonal)
+        const bool warp_ok = __all_sync(0xffffffffu, got);
+        const bool masked = (t == 0) || !valid;
+        const int lim = valid ? r : -1;
+        float rraw = NEG_INF;
+        if (warp_ok) {
 #pragma unroll
-          for (int cc = 0; cc < 4; ++cc) tmem_ld32(tS + cc * 32, v[cc]);
-          tmem_wait_ld();
-        } else {
+          for (int hh = 0; hh < 2; ++hh) {
+            uint32_t v[2][32];
+            tmem_ld32(tS + hh * 64, v[0]);
+            tmem_ld32(tS + hh * 64 + 32, v[1]);
+            tmem_wait_ld();
+            if (masked) {
 #pragma unroll
-          for (int cc = 0; cc < 4; ++cc)
+              for (int a = 0; a < 2; ++a)
 #pragma unroll
-            for (int e = 0; e < 32; ++e) v[cc][e] = 0xff800000u;  // -inf
-        }
-        float rmax = NEG_INF;
-        if (t == 0 || !valid) {
-          const int lim = valid ? r : -1;  // diagonal tile: keys c <= r are legal
+                for (int e = 0; e < 32; ++e) {
+                  const int col = hh * 64 + a * 32 + e;
+                  rraw = fmaxf(rraw, col <= lim ? __uint_as_float(v[a][e]) : NEG_INF);
+                }
+            } else {
 #pragma unroll
-          for (int cc = 0; cc < 4; ++cc)
+              for (int a = 0; a < 2; ++a)
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              float x = __uint_as_float(v[cc][e]) * p.scale_log2;
-              x = (cc * 32 + e <= lim) ? x : NEG_INF;
-              v[cc][e] = __float_as_uint(x);
-              rmax = fmaxf(rmax, x);
+                for (int e = 0; e < 32; ++e) rraw = fmaxf(rraw, __uint_as_float(v[a][e]));
             }
-        } else {
-#pragma unroll
-          for (int cc = 0; cc < 4; ++cc)
-#pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              const float x = __uint_as_float(v[cc][e]) * p.scale_log2;
-              v[cc][e] = __float_as_uint(x);
-              rmax = fmaxf(rmax, x);
-            }
+          }
         }
+        const float rmax = rraw * p.scale_log2;
         bool keep = true;
         if (kScreen) {
           const bool mine = (rmax != NEG_INF) && (l == 0.f || rmax >= m2 + __log2f(l) + thr2);
@@ -385,14 +383,27 @@ __global__ void __launch_bounds__(384, 1)
             tmem_st32(tO + cc * 32, o);
           }
         }
+        // pass 2: P = exp2(s * scale * log2(e) - m), 32 keys at a time, packed into the
+        // first 64 columns of the same TMEM region (each store lands on columns this
+        // thread has already read)
         float psum = 0.f;
 #pragma unroll
         for (int cc = 0; cc < 4; ++cc) {
+          uint32_t v[32];
+          if (warp_ok) {
+            tmem_ld32(tS + cc * 32, v);
+            tmem_wait_ld();
+          }
+          if (masked) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+              if (cc * 32 + e > lim) v[e] = 0xff800000u;  // -inf: P = 0
+          }
           uint32_t pk[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
-            const float p0 = fast_exp2(__uint_as_float(v[cc][2 * e]) - m_use);
-            const float p1 = fast_exp2(__uint_as_float(v[cc][2 * e + 1]) - m_use);
+            const float p0 = fast_exp2(fmaf(__uint_as_float(v[2 * e]), p.scale_log2, -m_use));
+            const float p1 = fast_exp2(fmaf(__uint_as_float(v[2 * e + 1]), p.scale_log2, -m_use));
             psum += p0 + p1;
             pk[e] = pack_bf16(p0, p1);
           }

@@ -80,16 +80,23 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
 
 // Waits for the phase with the given parity to complete.  Returns false (and flags the
 // CTA) when the budget runs out or another role of this CTA has already given up.
+// The abort flag and the clock are checked only every 256 polls, so that a waiting
+// thread notices a completed phase within a few cycles.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const AbortState& st,
                                           uint32_t site) {
   if (mbar_test(bar, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
-  while (true) {
+  uint64_t t0 = 0;
+  for (uint32_t it = 1;; ++it) {
     if (mbar_test(bar, parity)) return true;
-    if (*st.flag) return false;
-    if (globaltimer_ns() - t0 > st.budget_ns) {
-      record_timeout(st, site);
-      return false;
+    if ((it & 255u) == 0) {
+      if (*st.flag) return false;
+      const uint64_t now = globaltimer_ns();
+      if (t0 == 0) {
+        t0 = now;
+      } else if (now - t0 > st.budget_ns) {
+        record_timeout(st, site);
+        return false;
+      }
     }
   }
 }
