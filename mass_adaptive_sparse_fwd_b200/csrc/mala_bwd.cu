@@ -102,6 +102,10 @@ struct BwdShared {
   uint32_t abort_flag;
 };
 
+// dynamic + static shared memory must fit the 227 KB per-block limit of sm_100
+static_assert(BwdCfg<128>::SMEM + sizeof(BwdShared) <= 232448, "backward smem budget");
+static_assert(BwdCfg<64>::SMEM + sizeof(BwdShared) <= 232448, "backward smem budget");
+
 struct BUnit {
   int b, g, j, ntiles;  // tiles = G heads x (T - j) query blocks
 };
@@ -466,13 +470,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         mbar_arrive(&sh.p_full);
         // dS^T = P^T o (dP^T - D) -> bf16, swizzled K-major rows in shared memory (the
         // softmax scale is applied to dK in the epilogue and to dQ in the final convert)
+        // dP^T of this tile was issued after the previous tile's dK / dQ MMAs, and MMAs
+        // complete in issue order, so its completion also frees the dS^T buffer
         const bool dp_ok = mbar_wait_warp(&sh.dp_full, nret & 1, ast, 22);
         ++nret;
-        // the dS^T buffer is free once the previous tile's dK / dQ MMAs completed
-        bool buf_ok = true;
-        if (ntile > 0) buf_ok = mbar_wait_warp(&sh.dq_full, (ntile - 1) & 1, ast, 23);
         tc_fence_after();
-        if (dp_ok && buf_ok) {
+        if (dp_ok) {
 #pragma unroll
           for (int a = 0; a < 2; ++a) {
             uint32_t dp[32];

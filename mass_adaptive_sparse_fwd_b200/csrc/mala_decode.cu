@@ -78,6 +78,9 @@ struct DecShared {
   uint32_t abort_flag;
 };
 
+static_assert(DecCfg<128>::SMEM + sizeof(DecShared) <= 232448, "decode smem budget");
+static_assert(DecCfg<64>::SMEM + sizeof(DecShared) <= 232448, "decode smem budget");
+
 __device__ __forceinline__ void ldmatrix_x4(uint32_t addr, uint32_t& r0, uint32_t& r1,
                                             uint32_t& r2, uint32_t& r3) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"

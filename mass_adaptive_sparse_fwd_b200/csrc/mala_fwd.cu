@@ -69,6 +69,9 @@ struct FwdShared {
   uint32_t abort_flag;
 };
 
+static_assert(FwdCfg<128>::SMEM + sizeof(FwdShared) <= 232448, "forward smem budget");
+static_assert(FwdCfg<64>::SMEM + sizeof(FwdShared) <= 232448, "forward smem budget");
+
 struct Unit {
   int b, g, i, h0;
   bool active[2];
