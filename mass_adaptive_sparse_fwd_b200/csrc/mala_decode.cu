@@ -12,10 +12,12 @@
 // Decode is bound by HBM bandwidth: every K byte must be read, and V bytes only for
 // retained tiles.  The retention decisions depend on Q and K alone, so the kernel
 // decides ahead of the P.V work and gates each V load on the decision:
-//   warp 4      K producer: streams K tiles of the CTA's units into a ring (TMA).
-//   warp 5      V producer: waits for the decision of each tile and loads V only when
+//   warp CW     K producer: streams K tiles of the CTA's units into a ring (TMA).
+//   warp CW+1   V producer: waits for the decision of each tile and loads V only when
 //               at least one head of the group retains it.
-//   warps 0-3   consumers: scores S = K_t q_g^T (mma.sync m16n8k16, heads padded to
+//   warps 0..CW-1  consumers (CW = 8 for d = 128, two per SM sub-partition, so one
+//               warp's dependent mma / shuffle / barrier chain hides another's):
+//               scores S = K_t q_g^T (mma.sync m16n8k16, heads padded to
 //               8 as the N dimension), per-head tile maxima, retention test, online
 //               softmax state and P_t; the P.V product of tile t is done LAG tiles
 //               later, when its V has had time to arrive.
@@ -39,7 +41,6 @@ int sm_count();
 
 namespace {
 
-constexpr int kDecThreads = 192;
 constexpr int kLag = 2;        // tiles between a decision and its P.V
 constexpr int kPR = kLag + 1;  // P / decision ring depth
 
@@ -47,6 +48,13 @@ template <int D>
 struct DecCfg {
   static constexpr int TILE_BYTES = kTile * D * 2;
   static constexpr int BOXES = D / 64;
+  // consumer warps: warp w scores keys [16 KB w, 16 KB (w+1)) of a tile and owns
+  // head-dim rows [16 MB w, 16 MB (w+1)) of O^T
+  static constexpr int CW = (D == 128) ? 8 : 4;
+  static constexpr int KB = kTile / (16 * CW);
+  static constexpr int MB = D / (16 * CW);
+  static constexpr int NT = 32 * CW;            // consumer threads
+  static constexpr int THREADS = NT + 64;       // + K producer warp + V producer warp
   static constexpr int NK = (D == 128) ? 3 : 6;
   static constexpr int NV = (D == 128) ? 3 : 6;
   static constexpr int SMEM = (NK + NV) * TILE_BYTES + 1024;
@@ -73,7 +81,7 @@ struct DecShared {
   __nv_bfloat16 P[kPR][8][kTile];     // P_t, rows = heads (>= G zero)
   float alpha[kPR][8];                // rescale of O at tile t, per head
   uint32_t keep[kPR];                 // bit h: head h retained tile t
-  float red[4][8];                    // per-warp partial max / sum
+  float red[8][8];                    // per-warp partial max / sum
   uint32_t last_flag;
   uint32_t abort_flag;
 };
@@ -110,22 +118,25 @@ __device__ __forceinline__ uint32_t tile_chunk_addr(uint32_t base, int r, int c)
   return base + (c >> 3) * 16384 + sw128_offset(r, c & 7);
 }
 
+// Units are numbered KV head fastest: CTAs that run side by side stream the same key
+// range of all H_kv heads, i.e. whole [H_kv, d] rows of the cache, which keeps DRAM
+// pages fully used (one head's keys are 2*d-byte pieces at a 2*H_kv*d-byte stride).
 __device__ __forceinline__ void unit_coords(const DecParams& p, int u, int& b, int& g, int& s,
                                             int& t_lo, int& t_hi) {
-  s = u % p.S;
-  const int bg = u / p.S;
-  g = bg % p.Hkv;
-  b = bg / p.Hkv;
+  g = u % p.Hkv;
+  s = (u / p.Hkv) % p.S;
+  b = u / (p.Hkv * p.S);
   t_lo = static_cast<int>(static_cast<long long>(s) * p.T / p.S);
   t_hi = static_cast<int>(static_cast<long long>(s + 1) * p.T / p.S);
 }
 
 template <int D, bool kScreen>
-__global__ void __launch_bounds__(kDecThreads, 1)
+__global__ void __launch_bounds__(DecCfg<D>::THREADS, 1)
     mala_decode_kernel(const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const DecParams p) {
   using C = DecCfg<D>;
   constexpr int NK = C::NK, NV = C::NV;
+  constexpr int CW = C::CW, KB = C::KB, MB = C::MB, NT = C::NT;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -137,11 +148,11 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   if (tid == 0) {
     for (int i = 0; i < NK; ++i) {
       mbar_init(&sh.k_full[i], 1);
-      mbar_init(&sh.k_empty[i], 4);
+      mbar_init(&sh.k_empty[i], CW);
     }
     for (int i = 0; i < NV; ++i) {
       mbar_init(&sh.v_full[i], 1);
-      mbar_init(&sh.v_empty[i], 4);
+      mbar_init(&sh.v_empty[i], CW);
     }
     for (int i = 0; i < kPR; ++i) {
       mbar_init(&sh.dec_full[i], 1);
@@ -153,7 +164,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   __syncthreads();
   const AbortState ast{&sh.abort_flag, p.err, p.budget_ns, 0x300u};
 
-  if (warp == 4) {
+  if (warp == CW) {
     // ------------------------------------------------------------------ K producer
     if (lane == 0) {
       tma_prefetch_desc(&tmK);
@@ -180,7 +191,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
           mbar_wait(&sh.k_full[cc % NK], (cc / NK) & 1, drain, 2);
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == CW + 1) {
     // ------------------------------------------------------------------ V producer
     if (lane == 0) {
       tma_prefetch_desc(&tmV);
@@ -221,7 +232,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     uint32_t kc = 0, vc = 0, n_glob = 0;
     bool ok = true;
     // zero the padded heads of P once (rows >= G are never written again)
-    for (int i = tid; i < kPR * 8 * kTile; i += 128) {
+    for (int i = tid; i < kPR * 8 * kTile; i += NT) {
       const int row = (i / kTile) % 8;
       if (row >= G) (&sh.P[0][0][0])[i] = __float2bfloat16(0.f);
     }
@@ -230,13 +241,13 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       unit_coords(p, u, b, g, s, t_lo, t_hi);
       const int nt = t_hi - t_lo;
       // query rows of the group -> shared, then the B fragments of S = K q^T
-      named_bar_sync(1, 128);
-      for (int i = tid; i < 8 * D; i += 128) {
+      named_bar_sync(1, NT);
+      for (int i = tid; i < 8 * D; i += NT) {
         const int hh = i / D, c = i % D;
         sh.qs[hh][c] = (hh < G) ? p.q[(static_cast<size_t>(b) * p.H + g * G + hh) * D + c]
                                 : __float2bfloat16(0.f);
       }
-      named_bar_sync(1, 128);
+      named_bar_sync(1, NT);
       uint32_t qb[D / 16][2];
 #pragma unroll
       for (int ks = 0; ks < D / 16; ++ks) {
@@ -248,8 +259,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       float m[4], l[4];
 #pragma unroll
       for (int hh = 0; hh < 4; ++hh) { m[hh] = NEG_INF; l[hh] = 0.f; }
-      // O^T accumulators: warp owns head-dim rows [w*D/4, (w+1)*D/4)
-      constexpr int MB = D / 64;  // 16-row blocks per warp
+      // O^T accumulators: warp owns head-dim rows [16 MB w, 16 MB (w+1))
       float acc[MB][4];
 #pragma unroll
       for (int mb = 0; mb < MB; ++mb)
@@ -263,14 +273,14 @@ __global__ void __launch_bounds__(kDecThreads, 1)
           const int kst = kc % NK;
           // A failed wait only raises the abort flag; the consumers leave the loop
           // together, right after their next named barrier.
-          const bool got = __all_sync(0xffffffffu, mbar_wait(&sh.k_full[kst], (kc / NK) & 1, ast, 10));
+          const bool got = mbar_wait_warp(&sh.k_full[kst], (kc / NK) & 1, ast, 10);
           // scores of this warp's 32 keys x 8 (padded) heads
-          float sc[2][4];
+          float sc[KB][4];
 #pragma unroll
-          for (int kb = 0; kb < 2; ++kb) {
+          for (int kb = 0; kb < KB; ++kb) {
 #pragma unroll
             for (int e = 0; e < 4; ++e) sc[kb][e] = 0.f;
-            const int row0 = warp * 32 + kb * 16;
+            const int row0 = warp * (16 * KB) + kb * 16;
             if (got) {
 #pragma unroll
               for (int ks = 0; ks < D / 16; ++ks) {
@@ -288,10 +298,10 @@ __global__ void __launch_bounds__(kDecThreads, 1)
           // scale into log2 units, mask keys past the end, per-head tile maxima
           float mx[2] = {NEG_INF, NEG_INF};
 #pragma unroll
-          for (int kb = 0; kb < 2; ++kb)
+          for (int kb = 0; kb < KB; ++kb)
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-              const int key = t * kTile + warp * 32 + kb * 16 + (lane >> 2) + (e >> 1) * 8;
+              const int key = t * kTile + warp * (16 * KB) + kb * 16 + (lane >> 2) + (e >> 1) * 8;
               float x = sc[kb][e] * p.scale_log2;
               x = (key < p.Nk) ? x : NEG_INF;
               sc[kb][e] = x;
@@ -306,15 +316,16 @@ __global__ void __launch_bounds__(kDecThreads, 1)
             sh.red[warp][lane * 2] = mx[0];
             sh.red[warp][lane * 2 + 1] = mx[1];
           }
-          named_bar_sync(1, 128);
+          named_bar_sync(1, NT);
           if (*ast.flag) { ok = false; break; }
           // retention test per head (Eq. 3 with L_0 = N_k), identical in every thread
           uint32_t keep = 0;
           float mnew[4], alpha[4];
 #pragma unroll
           for (int hh = 0; hh < 4; ++hh) {
-            const float tmax = fmaxf(fmaxf(sh.red[0][hh], sh.red[1][hh]),
-                                     fmaxf(sh.red[2][hh], sh.red[3][hh]));
+            float tmax = sh.red[0][hh];
+#pragma unroll
+            for (int ww = 1; ww < CW; ++ww) tmax = fmaxf(tmax, sh.red[ww][hh]);
             bool k = hh < G;
             if (kScreen && k) k = (l[hh] == 0.f) || (tmax >= m[hh] + __log2f(l[hh]) + p.thr2);
             mnew[hh] = m[hh];
@@ -343,10 +354,10 @@ __global__ void __launch_bounds__(kDecThreads, 1)
             float ps[2] = {0.f, 0.f};
             const int h0 = (lane & 3) * 2;
 #pragma unroll
-            for (int kb = 0; kb < 2; ++kb)
+            for (int kb = 0; kb < KB; ++kb)
 #pragma unroll
               for (int r8 = 0; r8 < 2; ++r8) {
-                const int key = warp * 32 + kb * 16 + (lane >> 2) + r8 * 8;
+                const int key = warp * (16 * KB) + kb * 16 + (lane >> 2) + r8 * 8;
 #pragma unroll
                 for (int c = 0; c < 2; ++c) {
                   const int hh = h0 + c;
@@ -364,23 +375,25 @@ __global__ void __launch_bounds__(kDecThreads, 1)
               ps[0] += __shfl_xor_sync(0xffffffffu, ps[0], o);
               ps[1] += __shfl_xor_sync(0xffffffffu, ps[1], o);
             }
-            named_bar_sync(1, 128);  // everyone has read sh.red (maxima)
+            named_bar_sync(1, NT);  // everyone has read sh.red (maxima)
             if (lane < 2) {
               sh.red[warp][lane * 2] = ps[0];
               sh.red[warp][lane * 2 + 1] = ps[1];
             }
             if (tid < 8) sh.alpha[slot][tid] = (tid < 4) ? alpha[tid] : 1.f;
-            named_bar_sync(1, 128);
+            named_bar_sync(1, NT);
 #pragma unroll
             for (int hh = 0; hh < 4; ++hh) {
               if ((keep >> hh) & 1u) {
-                const float tsum = sh.red[0][hh] + sh.red[1][hh] + sh.red[2][hh] + sh.red[3][hh];
+                float tsum = 0.f;
+#pragma unroll
+                for (int ww = 0; ww < CW; ++ww) tsum += sh.red[ww][hh];
                 l[hh] = l[hh] * alpha[hh] + tsum;
                 m[hh] = mnew[hh];
               }
             }
           }
-          named_bar_sync(1, 128);  // sh.red is reused by the next tile
+          named_bar_sync(1, NT);  // sh.red is reused by the next tile
           if (*ast.flag) { ok = false; break; }
         }
         // P.V of the tile decided kLag iterations ago
@@ -390,8 +403,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
           const uint32_t keep2 = sh.keep[slot2];
           if (keep2) {
             const int vst = vc % NV;
-            const bool vgot =
-                __all_sync(0xffffffffu, mbar_wait(&sh.v_full[vst], (vc / NV) & 1, ast, 12));
+            const bool vgot = mbar_wait_warp(&sh.v_full[vst], (vc / NV) & 1, ast, 12);
             // rescale: thread's accumulator columns are heads (lane&3)*2 + {0,1}
             const int h0 = (lane & 3) * 2;
             const float a0 = (h0 < 4) ? sh.alpha[slot2][h0] : 1.f;
@@ -408,7 +420,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
               const uint32_t b1 = *reinterpret_cast<const uint32_t*>(&sh.P[slot2][hh][kk + 8]);
 #pragma unroll
               for (int mb = 0; mb < MB; ++mb) {
-                const int d0 = warp * (D / 4) + mb * 16;
+                const int d0 = warp * (16 * MB) + mb * 16;
                 const int mi = lane >> 3;
                 uint32_t r0, r1, r2, r3;
                 ldmatrix_x4_trans(
@@ -427,7 +439,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       }
       if (!ok) break;
       n_glob += nt;
-      named_bar_sync(1, 128);
+      named_bar_sync(1, NT);
       if (*ast.flag) { ok = false; break; }
       // this split's normalised output o_s = acc / l and z_s = (m + log2 l) ln 2
       {
@@ -437,7 +449,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int hh = h0 + (e & 1);
-            const int dd = warp * (D / 4) + mb * 16 + (lane >> 2) + (e >> 1) * 8;
+            const int dd = warp * (16 * MB) + mb * 16 + (lane >> 2) + (e >> 1) * 8;
             if (hh < G) {
               const float lv = (hh == 0) ? l[0] : (hh == 1) ? l[1] : (hh == 2) ? l[2] : l[3];
               p.part_o[((static_cast<size_t>(b) * p.H + g * G + hh) * p.S + s) * D + dd] =
@@ -449,16 +461,16 @@ __global__ void __launch_bounds__(kDecThreads, 1)
               (m[tid] + __log2f(l[tid])) * kLn2;
       }
       // last CTA of this (b, g) merges the splits
-      named_bar_sync(1, 128);
+      named_bar_sync(1, NT);
       if (tid == 0) {
         __threadfence();
         const uint32_t prev = atomicAdd(&p.tickets[b * p.Hkv + g], 1u);
         sh.last_flag = (prev == static_cast<uint32_t>(p.S - 1)) ? 1u : 0u;
       }
-      named_bar_sync(1, 128);
+      named_bar_sync(1, NT);
       if (sh.last_flag) {
         __threadfence();
-        for (int i = tid; i < G * D; i += 128) {
+        for (int i = tid; i < G * D; i += NT) {
           const int hh = i / D, dd = i % D;
           const size_t row = static_cast<size_t>(b) * p.H + g * G + hh;
           const volatile float* pz = p.part_z + row * p.S;
@@ -512,7 +524,7 @@ static cudaError_t launch_decode(const CUtensorMap& tk, const CUtensorMap& tv,
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        DecCfg<D>::SMEM);
   if (e != cudaSuccess) return e;
-  kern<<<grid, kDecThreads, DecCfg<D>::SMEM, stream>>>(tk, tv, p);
+  kern<<<grid, DecCfg<D>::THREADS, DecCfg<D>::SMEM, stream>>>(tk, tv, p);
   return cudaGetLastError();
 }
 
