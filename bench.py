@@ -35,7 +35,7 @@ sys.path.insert(0, ROOT)
 from mass_adaptive_sparse_fwd_b200 import synth  # noqa: E402
 
 METRIC = "MALA fwd+bwd ms and TFLOPS at 32K, decode µs at 128K; % of bf16 tensor peak"
-TRAIN = "sinkband32k"
+TRAIN = "sinkband32k"  # --train sinkband128k times the 128K one-GPU training shape instead
 DECODE = "decode128k"
 TAU = 1.0
 KERNELS_PER_STEP = 5  # fwd 1, bwd 3 (D preprocess, main, dQ convert), decode 1
@@ -219,7 +219,7 @@ def oracle_sample(wt: synth.Workload, wd: synth.Workload, train, dec, S: int,
     full_ms = 1e3 * ((t1 - t0) / fwd_tiles * legal + (t2 - t1) / bwd_tiles * 2 * legal +
                      (t3 - t2) / len(dunits) * wd.B * wd.H)
     desc = (f"oracle fp64 on {fwd_units} forward query blocks, {kv_units} dK/dV key blocks, "
-            f"{q_units} dQ query blocks of {TRAIN} and {len(dunits)} of {wd.B * wd.H} decode "
+            f"{q_units} dQ query blocks of {wt.name} and {len(dunits)} of {wd.B * wd.H} decode "
             f"rows of {DECODE}; extrapolated to the full step by tile / row counts")
     return full_ms, t3 - t0, desc
 
@@ -265,7 +265,7 @@ def run_mala(args, dist: Dist):
     dev = torch.device("cuda", dist.local_rank)
     torch.cuda.set_device(dev)
     peaks = _peaks()
-    wt = rank_workload(synth.WORKLOADS[TRAIN], dist.rank)
+    wt = rank_workload(synth.WORKLOADS[args.train], dist.rank)
     wd = rank_workload(synth.WORKLOADS[DECODE], dist.rank)
     train = synth.make_training(wt)
     dec = synth.make_decode(wd)
@@ -439,8 +439,9 @@ def run_mala(args, dist: Dist):
             "ms_per_step": res["step_ms"], "higher_is_better": False, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded generator; states stand in for real model states)",
-            "config": {"workload": f"{TRAIN} fwd+bwd (B=1,H=32,H_kv=8,L=32768,d=128) + "
-                                   f"{DECODE} decode (B=4,H=32,H_kv=8,N_k=131072,d=128)",
+            "config": {"workload": f"{args.train} fwd+bwd (B={wt.B},H={wt.H},H_kv={wt.H_kv},"
+                                   f"L={wt.L},d={wt.d}) + {DECODE} decode "
+                                   "(B=4,H=32,H_kv=8,N_k=131072,d=128)",
                        "tau": TAU, "decode_splits": S,
                        "l2": "inputs larger than L2 (Q 268 MB, dO 268 MB, KV cache 2.1 GB)",
                        "parallelism": f"weak: {dist.world} independent problem(s), one per GPU"},
@@ -481,6 +482,8 @@ def main():
     ap.add_argument("--impl", choices=("mala", "reference"), default="mala")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--train", default=TRAIN, choices=("sinkband32k", "sinkband128k"),
+                    help="training workload of the step (default: the 32K headline shape)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

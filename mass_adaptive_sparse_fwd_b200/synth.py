@@ -24,6 +24,8 @@ available; these synthetic distributions stand in for them):
 * ``decode128k``  B=4, H=32, H_kv=8, N_k=131072, d=128, bf16; K, V, q ~ N(0, 1); per
                   (b, KV head) 16 distinct random positions get a planted key
                   3.0 * sqrt(d) * q_h / |q_h| + N(0, 1), h cycling over the group's heads
+* ``sinkband128k`` B=1, H=8, H_kv=1, L=131072, d=128, bf16; sink + band states as
+                  ``sinkband32k`` (one rank of an 8-way head-sharded 64/8-head model)
 
 V ~ N(0, 1) everywhere; dO is a Rademacher (+-1) probe.
 """
@@ -68,6 +70,9 @@ WORKLOADS = {
     "sinkband32k": Workload("sinkband32k", 1, 32, 8, 32768, 128, "bf16", "sink_band", 3),
     "decode128k": Workload("decode128k", 4, 32, 8, 131072, 128, "bf16", "planted", 4,
                            decode=True),
+    # 128K-token training on one GPU: the per-rank shape of a 64-query-head / 8-KV-head
+    # model under 8-way head sharding, with the sink + band states of sinkband32k
+    "sinkband128k": Workload("sinkband128k", 1, 8, 1, 131072, 128, "bf16", "sink_band", 5),
 }
 
 

@@ -132,3 +132,11 @@ def test_bwd_tiny256_fp32(orc, mala, tau):
 def test_bwd_fp32_ragged_gqa(orc, mala):
     w, inp = synth.small_training(B=2, H=4, Hkv=2, L=200, d=32, dtype="fp32", structure="peaked")
     check_bwd(orc, mala, w, inp, 1.0)
+
+
+@pytest.mark.slow
+def test_bwd_sinkband128k_sampled(orc, mala):
+    w = synth.WORKLOADS["sinkband128k"]
+    T = w.L // 128
+    check_bwd(orc, mala, w, synth.make_training(w), 1.0,
+              kv_units=[(0, 0, T - 2)], q_units=[(0, 6, T - 1), (0, 1, 3)])

@@ -113,3 +113,11 @@ def test_fwd_tiny256_fp32(orc, mala, tau):
 def test_fwd_fp32_ragged_gqa(orc, mala):
     w, inp = synth.small_training(B=2, H=4, Hkv=2, L=200, d=32, dtype="fp32", structure="peaked")
     check_fwd(orc, mala, w, inp, 1.0)
+
+
+@pytest.mark.slow
+def test_fwd_sinkband128k_sampled(orc, mala):
+    w = synth.WORKLOADS["sinkband128k"]
+    inp = synth.make_training(w)
+    T = w.L // 128
+    check_fwd(orc, mala, w, inp, 1.0, units=[(0, 7, T - 1), (0, 0, T // 3), (0, 3, 2)])
