@@ -36,6 +36,7 @@ from mass_adaptive_sparse_fwd_b200 import synth  # noqa: E402
 
 METRIC = "MALA fwd+bwd ms and TFLOPS at 32K, decode µs at 128K; % of bf16 tensor peak"
 TRAIN = "sinkband32k"  # --train sinkband128k times the 128K one-GPU training shape instead
+SKIP_TRAIN = "prevtok32k"  # concentrated states for the skip-regime block
 DECODE = "decode128k"
 TAU = 1.0
 KERNELS_PER_STEP = 5  # fwd 1, bwd 3 (D preprocess, main, dQ convert), decode 1
@@ -425,6 +426,77 @@ def run_mala(args, dist: Dist):
                "note": "fwd+bwd+decode step incl. host->device inputs (Q,K,V,dO,q; the KV "
                        "cache is resident) and device->host outputs"}
 
+    # skip regime: the same fwd + bwd on concentrated "previous-token" states, where most
+    # tiles fall below tau / L_q; shows the step time following the retained work
+    skip = None
+    if not args.no_skip_regime:
+        wl = rank_workload(synth.WORKLOADS[SKIP_TRAIN], dist.rank)
+        loc = synth.make_training(wl)
+        sQ, sK, sV, sdO = (bf(loc[k]) for k in ("Q", "K", "V", "dO"))
+        del loc
+        sO = torch.empty_like(sQ)
+        sLSE = torch.empty((wl.B, wl.H, wl.L), dtype=torch.float32, device=dev)
+        sdQ, sdK, sdV = torch.empty_like(sQ), torch.empty_like(sK), torch.empty_like(sV)
+        swf = mala.alloc_workspace(mala.fwd_workspace_bytes(wl.B, wl.H, wl.H_kv, wl.L, wl.d), dev)
+        swb = mala.alloc_workspace(mala.bwd_workspace_bytes(wl.B, wl.H, wl.H_kv, wl.L, wl.d), dev)
+
+        def sfwd(tau, mask=None):
+            mala.mala_fwd(sQ, sK, sV, wl.scale, tau, O=sO, LSE=sLSE, workspace=swf, tile_mask=mask)
+
+        def sbwd(tau, mask=None):
+            mala.mala_bwd(sQ, sK, sV, sO, sLSE, sdO, wl.scale, tau, dQ=sdQ, dK=sdK, dV=sdV,
+                          workspace=swb, tile_mask=mask)
+
+        def fb(tau):
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+            for _ in range(args.warmup):
+                sfwd(tau)
+                sbwd(tau)
+            torch.cuda.synchronize(dev)
+            dist.barrier()
+            torch.cuda.synchronize(dev)
+            ev[0].record(stream)
+            for _ in range(args.steps):
+                sfwd(tau)
+            ev[1].record(stream)
+            for _ in range(args.steps):
+                sbwd(tau)
+            ev[2].record(stream)
+            torch.cuda.synchronize(dev)
+            dist.barrier()
+            for ws in (swf, swb):
+                err = mala.read_device_error(ws)
+                if err:
+                    raise RuntimeError(f"device error word 0x{err:x}")
+            return (dist.max(ev[0].elapsed_time(ev[1]) / args.steps, device=dev),
+                    dist.max(ev[1].elapsed_time(ev[2]) / args.steps, device=dev))
+
+        sf1, sb1 = fb(TAU)
+        sf0, sb0 = fb(0.0)
+        sT = mala.n_tiles(wl.L)
+        sfm = torch.zeros((wl.B, wl.H, sT, sT), dtype=torch.uint8, device=dev)
+        sbm = torch.zeros_like(sfm)
+        sfwd(TAU, sfm)
+        sbwd(TAU, sbm)
+        torch.cuda.synchronize(dev)
+        slegal = torch.ones(sT, sT, dtype=torch.bool, device=dev).tril()
+        sfr = float(sfm[:, :, slegal].float().mean())
+        sbr = float(sbm[:, :, slegal].float().mean())
+        sfl = fwd_bwd_flops(wl, sfr, sbr)
+        sfl0 = fwd_bwd_flops(wl, 1.0, 1.0)
+        skip = {"workload": f"{SKIP_TRAIN} (B={wl.B},H={wl.H},H_kv={wl.H_kv},L={wl.L},d={wl.d}; "
+                            "q_t = 18 sqrt(d) K_(t-1) / |K_(t-1)|^2 + 0.3 noise)",
+                "retained": {"fwd_tiles": sfr, "bwd_tiles": sbr},
+                "tau1": {"fwd_ms": sf1, "bwd_ms": sb1, "fwd_bwd_ms": sf1 + sb1,
+                         "executed_tflops": (sfl["fwd_exec"] + sfl["bwd_exec"]) /
+                                            ((sf1 + sb1) * 1e-3) / 1e12},
+                "tau0": {"fwd_ms": sf0, "bwd_ms": sb0, "fwd_bwd_ms": sf0 + sb0},
+                "speedup_vs_tau0": {"fwd": sf0 / sf1, "bwd": sb0 / sb1,
+                                    "fwd_bwd": (sf0 + sb0) / (sf1 + sb1)},
+                "work_ratio": {"fwd": sfl["fwd_exec"] / sfl0["fwd_exec"],
+                               "bwd": sfl["bwd_exec"] / sfl0["bwd_exec"]}}
+        del sQ, sK, sV, sdO, sO, sLSE, sdQ, sdK, sdV, swf, swb
+
     cpu = None
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
         ms, spent, desc = oracle_sample(wt, wd, train, dec, S)
@@ -470,6 +542,7 @@ def run_mala(args, dist: Dist):
             "gpu_launches": KERNELS_PER_STEP * args.steps,
             "e2e": e2e,
             "cpu_baseline": cpu,
+            "skip_regime": skip,
         }
         print(json.dumps(line), flush=True)
 
@@ -482,6 +555,7 @@ def main():
     ap.add_argument("--impl", choices=("mala", "reference"), default="mala")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-skip-regime", action="store_true")
     ap.add_argument("--train", default=TRAIN, choices=("sinkband32k", "sinkband128k"),
                     help="training workload of the step (default: the 32K headline shape)")
     args = ap.parse_args()

@@ -26,6 +26,10 @@ available; these synthetic distributions stand in for them):
                   3.0 * sqrt(d) * q_h / |q_h| + N(0, 1), h cycling over the group's heads
 * ``sinkband128k`` B=1, H=8, H_kv=1, L=131072, d=128, bf16; sink + band states as
                   ``sinkband32k`` (one rank of an 8-way head-sharded 64/8-head model)
+* ``prevtok32k``  B=1, H=32, H_kv=8, L=32768, d=128, bf16; concentrated "previous-token"
+                  heads: q_t = 18 sqrt(d) K_{t-1} / |K_{t-1}|^2 + 0.3 N(0, 1), so the
+                  previous token's scaled score is ~18 and the rest of the row is a flat
+                  tail of 1e-5 .. 2e-3 of the mass (most off-diagonal tiles skippable)
 
 V ~ N(0, 1) everywhere; dO is a Rademacher (+-1) probe.
 """
@@ -73,6 +77,9 @@ WORKLOADS = {
     # 128K-token training on one GPU: the per-rank shape of a 64-query-head / 8-KV-head
     # model under 8-way head sharding, with the sink + band states of sinkband32k
     "sinkband128k": Workload("sinkband128k", 1, 8, 1, 131072, 128, "bf16", "sink_band", 5),
+    # concentrated heads: each query copies the previous token's key (a "previous-token"
+    # head), so most off-diagonal tiles fall below tau / L_q and are skipped
+    "prevtok32k": Workload("prevtok32k", 1, 32, 8, 32768, 128, "bf16", "prev_token", 6),
 }
 
 
@@ -182,6 +189,20 @@ def make_training(w: Workload, L: int | None = None) -> dict:
         Q = np.empty((B, L, H, d), dtype=np.float32)
         for h in range(H):
             Q[:, :, h] = 0.5 * u[:, :, h // G] + math.sqrt(0.75) * n[:, :, h]
+        Q = _round(Q, w.dtype)
+    elif w.structure == "prev_token":
+        # q_t = s0 sqrt(d) K_{t-1} / |K_{t-1}|^2 + b n_t: the scaled score of the previous
+        # token is s0 (up to the noise) for every row, the other scores spread with a
+        # standard deviation near s0 / |K| + b, so each head puts all but a small, flat tail
+        # of its mass on the previous token (q_0 = b n_0)
+        s0, b = 18.0, 0.3
+        n = normal(w.seed, _NOISE, (B, L, H, d), "fp32")
+        G = H // Hkv
+        kp = K[:, :-1].astype(np.float64)
+        kp = kp * (s0 * math.sqrt(d) / np.maximum((kp * kp).sum(-1, keepdims=True), 1e-6))
+        Q = b * n
+        for h in range(H):
+            Q[:, 1:, h] += kp[:, :, h // G].astype(np.float32)
         Q = _round(Q, w.dtype)
     else:
         raise ValueError(w.structure)

@@ -140,3 +140,18 @@ def test_bwd_sinkband128k_sampled(orc, mala):
     T = w.L // 128
     check_bwd(orc, mala, w, synth.make_training(w), 1.0,
               kv_units=[(0, 0, T - 2)], q_units=[(0, 6, T - 1), (0, 1, 3)])
+
+
+def test_bwd_prev_token_skips(orc, mala):
+    w, inp = synth.small_training(B=1, H=4, Hkv=1, L=2048, d=128, structure="prev_token", seed=3)
+    st = check_bwd(orc, mala, w, inp, 1.0)
+    assert st["bwd_retained"] < 0.3
+
+
+@pytest.mark.slow
+def test_bwd_prevtok32k_sampled(orc, mala):
+    w = synth.WORKLOADS["prevtok32k"]
+    T = w.L // 128
+    st = check_bwd(orc, mala, w, synth.make_training(w), 1.0,
+                   kv_units=[(0, 5, T - 3), (0, 0, 7)], q_units=[(0, 31, T - 1), (0, 2, 40)])
+    assert st["bwd_retained"] < 0.05

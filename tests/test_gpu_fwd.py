@@ -121,3 +121,19 @@ def test_fwd_sinkband128k_sampled(orc, mala):
     inp = synth.make_training(w)
     T = w.L // 128
     check_fwd(orc, mala, w, inp, 1.0, units=[(0, 7, T - 1), (0, 0, T // 3), (0, 3, 2)])
+
+
+def test_fwd_prev_token_skips(orc, mala):
+    """Concentrated heads: most off-diagonal tiles are skipped; decisions and O agree."""
+    w, inp = synth.small_training(B=1, H=4, Hkv=1, L=2048, d=128, structure="prev_token", seed=3)
+    st = check_fwd(orc, mala, w, inp, 1.0)
+    assert st["retained"] < 0.3
+
+
+@pytest.mark.slow
+def test_fwd_prevtok32k_sampled(orc, mala):
+    w = synth.WORKLOADS["prevtok32k"]
+    inp = synth.make_training(w)
+    T = w.L // 128
+    st = check_fwd(orc, mala, w, inp, 1.0, units=_units(w.B, w.H, T, 6, seed=9))
+    assert st["retained"] < 0.05
