@@ -92,7 +92,7 @@ struct BwdShared {
   // per softmax warpgroup and query column: LSE_q in log2 units (+inf past L, so the
   // probability is 0 there), the threshold log2(tau / L_q) and D_q
   alignas(16) float lse2[2][64];
-  alignas(16) float thr2[2][64];
+  alignas(16) float cut2[2][64];  // LSE2_q + log2(tau / L_q): the screen's cut
   alignas(16) float dsum[2][64];
   int sched_ring[2];
   uint32_t dec;      // decision of the current tile (1 = retained)
@@ -161,11 +161,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     mbar_init(&sh.do_full, 1);
     mbar_init(&sh.do_empty, 1);
     mbar_init(&sh.s_full, 1);
-    mbar_init(&sh.p_full, 256);
+    mbar_init(&sh.p_full, 8);   // one arrival per softmax warp
     mbar_init(&sh.dp_full, 1);
-    mbar_init(&sh.ds_full, 256);
+    mbar_init(&sh.ds_full, 8);
     mbar_init(&sh.dq_full, 1);
-    mbar_init(&sh.dq_empty, 128);
+    mbar_init(&sh.dq_empty, 4);  // one arrival per drain warp
     mbar_init(&sh.acc_full, 1);
     mbar_init(&sh.acc_empty, 128);
     for (int s = 0; s < 2; ++s) {
@@ -281,6 +281,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           if (!(ok = mbar_wait(&sh.p_full, ntile & 1, ast, 13))) break;
           tc_fence_after();
           const bool keep = sh.dec != 0;
+          // a skipped tile's Q stage was read only by its S^T MMA, which has completed:
+          // release it now so that the producer's next Q load starts a step earlier
+          if (!keep) umma_commit(&sh.q_empty[st]);
           // dO(c) is loaded for every tile; its stage is released after dP^T / dV
           if (!(ok = mbar_wait(&sh.do_full, c & 1, ast, 20))) break;
           if (keep) {
@@ -334,7 +337,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           if (ntile > 0 && !(ok = mbar_wait(&sh.dq_empty, (ntile - 1) & 1, ast, 19))) break;
           sh.dq_flag[ntile & 1] = keep ? 1u : 0u;
           umma_commit(&sh.dq_full);
-          umma_commit(&sh.q_empty[st]);
+          if (keep) umma_commit(&sh.q_empty[st]);  // after dK has read Q_i
         }
         if (!ok) break;
         if (!acc_waited && !(ok = acc_waited = mbar_wait(&sh.acc_empty, (nu - 1) & 1, ast, 15)))
@@ -371,33 +374,34 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const BUnit w = decode_bunit(p, u);
       const int krow = w.j * kTile + r;
       const bool kvalid = krow < p.L;
-      // per-column constants (LSE in log2 units, threshold, D) of tile n, loaded one tile
-      // ahead into registers by threads tw < 64 and published through shared memory
-      auto load_cols = [&](int n, float& l2, float& t2, float& ds) {
+      // per-column constants (LSE in log2 units, the screen's cut LSE2 + log2(tau / L_q),
+      // D) of tile n, loaded one tile ahead into registers by threads tw < 64 and
+      // published through shared memory
+      auto load_cols = [&](int n, float& l2, float& c2, float& ds) {
         int h, i;
         tile_hi(p, w, n, h, i);
         const int q = i * kTile + wg * 64 + tw;
-        l2 = INFINITY; t2 = INFINITY; ds = 0.f;
+        l2 = INFINITY; c2 = INFINITY; ds = 0.f;
         if (tw < 64 && q < p.L) {
           const size_t idx = (static_cast<size_t>(w.b) * p.H + h) * p.L + q;
           l2 = p.LSE[idx] * kLog2e;
           ds = p.Dsum[idx];
-          t2 = kScreen ? p.log2_tau - __log2f(static_cast<float>(q + 1)) : NEG_INF;
+          if (kScreen) c2 = l2 + (p.log2_tau - __log2f(static_cast<float>(q + 1)));
         }
       };
-      float nl2, nt2, nds;
-      load_cols(0, nl2, nt2, nds);
+      float nl2, nc2, nds;
+      load_cols(0, nl2, nc2, nds);
       for (int n = 0; n < w.ntiles; ++n, ++ntile) {
         int h, i;
         tile_hi(p, w, n, h, i);
         named_bar_sync(2 + wg, 128);  // previous tile's readers are done
         if (tw < 64) {
           sh.lse2[wg][tw] = nl2;
-          sh.thr2[wg][tw] = nt2;
+          sh.cut2[wg][tw] = nc2;
           sh.dsum[wg][tw] = nds;
         }
         named_bar_sync(2 + wg, 128);
-        if (n + 1 < w.ntiles) load_cols(n + 1, nl2, nt2, nds);
+        if (n + 1 < w.ntiles) load_cols(n + 1, nl2, nc2, nds);
         const bool got = mbar_wait_warp(&sh.s_full, ntile & 1, ast, 21);
         tc_fence_after();
         uint32_t v[2][32];
@@ -411,53 +415,74 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
             for (int e = 0; e < 32; ++e) v[a][e] = 0xff800000u;
         }
-        // a = log2 P = s * scale * log2(e) - LSE2_q (-inf past L through LSE2 = +inf);
-        // the tile is kept if some legal entry has a >= log2(tau / L_q) (Eq. 4).
-        // Causal masking is needed only on the diagonal block and past the last key.
-        // local column must be >= qlo: -1 off the diagonal, 64 for key rows past the end
+        // log2 P = s * scale * log2(e) - LSE2_q (-inf past L through LSE2 = +inf); the
+        // tile is kept if some legal entry has log2 P >= log2(tau / L_q) (Eq. 4), i.e.
+        // s * scale * log2(e) - cut2_q >= 0 with cut2_q = LSE2_q + log2(tau / L_q).
+        // Causal masking is needed only on the diagonal block and past the last key:
+        // the local column must be >= qlo (-1 off the diagonal, 64 for rows past L).
         const int qlo = !kvalid ? 64 : (i == w.j ? r - wg * 64 : -1);
-        float ymax = NEG_INF;
-        const float4* l4 = reinterpret_cast<const float4*>(sh.lse2[wg]);
-        const float4* t4 = reinterpret_cast<const float4*>(sh.thr2[wg]);
-#pragma unroll
-        for (int a = 0; a < 2; ++a)
-#pragma unroll
-          for (int e4 = 0; e4 < 8; ++e4) {
-            const float4 lv = l4[a * 8 + e4];
-            const float4 tv = t4[a * 8 + e4];
-            const float lq[4] = {lv.x, lv.y, lv.z, lv.w};
-            const float tq[4] = {tv.x, tv.y, tv.z, tv.w};
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-              const int cl = a * 32 + e4 * 4 + c;
-              float x = fmaf(__uint_as_float(v[a][e4 * 4 + c]), p.scale_log2, -lq[c]);
-              x = (cl >= qlo) ? x : NEG_INF;
-              v[a][e4 * 4 + c] = __float_as_uint(x);
-              if (kScreen) ymax = fmaxf(ymax, x - tq[c]);
-            }
-          }
         bool keep = true;
-        if (kScreen) keep = named_bar_or(1, 256, ymax >= 0.f);
-        else named_bar_sync(1, 256);  // every S^T load done before P overwrites it
+        if (kScreen) {
+          const float4* c4 = reinterpret_cast<const float4*>(sh.cut2[wg]);
+          float ymax = NEG_INF;
+          if (qlo < 0) {
+#pragma unroll
+            for (int a = 0; a < 2; ++a)
+#pragma unroll
+              for (int e4 = 0; e4 < 8; ++e4) {
+                const float4 cv = c4[a * 8 + e4];
+                const uint32_t* sv = &v[a][e4 * 4];
+                const float y0 = fmaf(__uint_as_float(sv[0]), p.scale_log2, -cv.x);
+                const float y1 = fmaf(__uint_as_float(sv[1]), p.scale_log2, -cv.y);
+                const float y2 = fmaf(__uint_as_float(sv[2]), p.scale_log2, -cv.z);
+                const float y3 = fmaf(__uint_as_float(sv[3]), p.scale_log2, -cv.w);
+                ymax = fmax3(ymax, y0, y1);
+                ymax = fmax3(ymax, y2, y3);
+              }
+          } else {
+#pragma unroll
+            for (int a = 0; a < 2; ++a)
+#pragma unroll
+              for (int e4 = 0; e4 < 8; ++e4) {
+                const float4 cv = c4[a * 8 + e4];
+                const float cq[4] = {cv.x, cv.y, cv.z, cv.w};
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                  const float y = fmaf(__uint_as_float(v[a][e4 * 4 + c]), p.scale_log2, -cq[c]);
+                  ymax = (a * 32 + e4 * 4 + c >= qlo) ? fmaxf(ymax, y) : ymax;
+                }
+              }
+          }
+          keep = named_bar_or(1, 256, ymax >= 0.f);
+        } else {
+          named_bar_sync(1, 256);  // every S^T load done before P overwrites it
+        }
         if (*ast.flag) { ok = false; break; }
         if (p.tile_mask && tid == 128)
           p.tile_mask[((static_cast<size_t>(w.b) * p.H + h) * p.T + i) * p.T + w.j] = keep ? 1 : 0;
         if (!keep) {
           if (tid == 128) sh.dec = 0;
           tc_fence_before();
-          mbar_arrive(&sh.p_full);
+          warp_arrive(&sh.p_full);
           continue;
         }
-        // P^T = exp2(a) -> bf16 pairs into TMEM columns [32 wg, 32 wg + 32)
+        // P^T = exp2(log2 P) -> bf16 pairs into TMEM columns [32 wg, 32 wg + 32)
         float pf[64];
+        const float4* l4 = reinterpret_cast<const float4*>(sh.lse2[wg]);
 #pragma unroll
         for (int a = 0; a < 2; ++a) {
           uint32_t pk[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
             const int c0 = a * 32 + 2 * e;
-            const float p0 = fast_exp2(__uint_as_float(v[a][2 * e]));
-            const float p1 = fast_exp2(__uint_as_float(v[a][2 * e + 1]));
+            const float4 lv = l4[c0 >> 2];
+            const float la = (e & 1) ? lv.z : lv.x, lb = (e & 1) ? lv.w : lv.y;
+            float x0 = fmaf(__uint_as_float(v[a][2 * e]), p.scale_log2, -la);
+            float x1 = fmaf(__uint_as_float(v[a][2 * e + 1]), p.scale_log2, -lb);
+            x0 = (c0 >= qlo) ? x0 : NEG_INF;
+            x1 = (c0 + 1 >= qlo) ? x1 : NEG_INF;
+            const float p0 = fast_exp2(x0);
+            const float p1 = fast_exp2(x1);
             pf[c0] = p0;
             pf[c0 + 1] = p1;
             pk[e] = pack_bf16(p0, p1);
@@ -467,7 +492,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tmem_wait_st();
         if (tid == 128) sh.dec = 1;
         tc_fence_before();
-        mbar_arrive(&sh.p_full);
+        warp_arrive(&sh.p_full);
         // dS^T = P^T o (dP^T - D) -> bf16, swizzled K-major rows in shared memory (the
         // softmax scale is applied to dK in the epilogue and to dQ in the final convert)
         // dP^T of this tile was issued after the previous tile's dK / dQ MMAs, and MMAs
@@ -501,7 +526,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
         fence_proxy_async_smem();
         tc_fence_before();
-        mbar_arrive(&sh.ds_full);
+        warp_arrive(&sh.ds_full);
       }
     }
   } else if (warp >= 12) {
@@ -528,7 +553,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const bool drain = named_bar_or(5, 128, got_dq && sh.dq_flag[ntile & 1] != 0);
         if (!drain) {
           tc_fence_before();
-          mbar_arrive(&sh.dq_empty);
+          warp_arrive(&sh.dq_empty);
           continue;
         }
         // dQ tile (row r of query block i): 64 columns per round through the staging
@@ -542,7 +567,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           tmem_wait_ld();
           if (half == D / 64 - 1) {
             tc_fence_before();
-            mbar_arrive(&sh.dq_empty);
+            warp_arrive(&sh.dq_empty);
           }
           // staging buffer free: the previous round's bulk reads have completed
           if (tid == 384) bulk_wait_read_all();
