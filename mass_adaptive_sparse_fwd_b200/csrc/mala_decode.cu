@@ -78,10 +78,15 @@ struct DecShared {
   uint64_t k_full[6], k_empty[6], v_full[6], v_empty[6];
   uint64_t dec_full[kPR], dec_empty[kPR];
   __nv_bfloat16 qs[8][128];           // query rows of the group, heads >= G are zero
-  __nv_bfloat16 P[kPR][8][kTile];     // P_t, rows = heads (>= G zero)
+  // P_t, rows = heads (>= G zero); rows padded by 8 keys so that the P.V fragment
+  // loads (8 heads x 4 key pairs per warp) fall on 32 distinct banks
+  __nv_bfloat16 P[kPR][8][kTile + 8];
   float alpha[kPR][8];                // rescale of O at tile t, per head
   uint32_t keep[kPR];                 // bit h: head h retained tile t
-  float red[8][8];                    // per-warp partial max / sum
+  // per-warp partial tile maxima of tile n and row sums of tile n - 1 (heads 0..3),
+  // double-buffered by the parity of n
+  float4 rmax[2][8];
+  float4 rsum[2][8];
   uint32_t last_flag;
   uint32_t abort_flag;
 };
@@ -232,8 +237,8 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, 1)
     uint32_t kc = 0, vc = 0, n_glob = 0;
     bool ok = true;
     // zero the padded heads of P once (rows >= G are never written again)
-    for (int i = tid; i < kPR * 8 * kTile; i += NT) {
-      const int row = (i / kTile) % 8;
+    for (int i = tid; i < kPR * 8 * (kTile + 8); i += NT) {
+      const int row = (i / (kTile + 8)) % 8;
       if (row >= G) (&sh.P[0][0][0])[i] = __float2bfloat16(0.f);
     }
     for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
@@ -255,10 +260,32 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, 1)
         qb[ks][0] = *reinterpret_cast<const uint32_t*>(&sh.qs[hh][c0]);
         qb[ks][1] = *reinterpret_cast<const uint32_t*>(&sh.qs[hh][c0 + 8]);
       }
-      // per-head running state (replicated in every consumer thread)
-      float m[4], l[4];
+      // per-head running state (replicated in every consumer thread).  The normaliser
+      // update of tile n (l = l alpha + row sum, m = mnew) is applied after the next
+      // barrier, which publishes the row sums; the test of tile n + 1 comes after it.
+      float m[4], l[4], palpha[4], pmnew[4];
+      float ps_prev[2] = {0.f, 0.f};  // this warp's row sums of the last decided tile
+      uint32_t pkeep = 0;
 #pragma unroll
-      for (int hh = 0; hh < 4; ++hh) { m[hh] = NEG_INF; l[hh] = 0.f; }
+      for (int hh = 0; hh < 4; ++hh) {
+        m[hh] = NEG_INF; l[hh] = 0.f; palpha[hh] = 1.f; pmnew[hh] = NEG_INF;
+      }
+      auto close_tile = [&](int rb) {
+        if (!pkeep) return;
+        float4 ts4 = sh.rsum[rb][0];
+#pragma unroll
+        for (int ww = 1; ww < CW; ++ww) {
+          const float4 v4 = sh.rsum[rb][ww];
+          ts4.x += v4.x; ts4.y += v4.y; ts4.z += v4.z; ts4.w += v4.w;
+        }
+        const float tsum[4] = {ts4.x, ts4.y, ts4.z, ts4.w};
+#pragma unroll
+        for (int hh = 0; hh < 4; ++hh)
+          if ((pkeep >> hh) & 1u) {
+            l[hh] = l[hh] * palpha[hh] + tsum[hh];
+            m[hh] = pmnew[hh];
+          }
+      };
       // O^T accumulators: warp owns head-dim rows [16 MB w, 16 MB (w+1))
       float acc[MB][4];
 #pragma unroll
@@ -312,20 +339,34 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, 1)
             mx[0] = fmaxf(mx[0], __shfl_xor_sync(0xffffffffu, mx[0], o));
             mx[1] = fmaxf(mx[1], __shfl_xor_sync(0xffffffffu, mx[1], o));
           }
+          // the tile's only barrier: this tile's per-warp maxima travel together with
+          // the previous tile's per-warp row sums
+          const int rb = n & 1;
           if (lane < 2) {  // lanes 0, 1 hold heads 0-1 and 2-3
-            sh.red[warp][lane * 2] = mx[0];
-            sh.red[warp][lane * 2 + 1] = mx[1];
+            float* rm = reinterpret_cast<float*>(&sh.rmax[rb][warp]);
+            float* rs = reinterpret_cast<float*>(&sh.rsum[rb][warp]);
+            rm[lane * 2] = mx[0];
+            rm[lane * 2 + 1] = mx[1];
+            rs[lane * 2] = ps_prev[0];
+            rs[lane * 2 + 1] = ps_prev[1];
           }
           named_bar_sync(1, NT);
           if (*ast.flag) { ok = false; break; }
+          if (n > 0) close_tile(rb);
           // retention test per head (Eq. 3 with L_0 = N_k), identical in every thread
+          float4 tm4 = sh.rmax[rb][0];
+#pragma unroll
+          for (int ww = 1; ww < CW; ++ww) {
+            const float4 v4 = sh.rmax[rb][ww];
+            tm4.x = fmaxf(tm4.x, v4.x); tm4.y = fmaxf(tm4.y, v4.y);
+            tm4.z = fmaxf(tm4.z, v4.z); tm4.w = fmaxf(tm4.w, v4.w);
+          }
+          const float tmx[4] = {tm4.x, tm4.y, tm4.z, tm4.w};
           uint32_t keep = 0;
           float mnew[4], alpha[4];
 #pragma unroll
           for (int hh = 0; hh < 4; ++hh) {
-            float tmax = sh.red[0][hh];
-#pragma unroll
-            for (int ww = 1; ww < CW; ++ww) tmax = fmaxf(tmax, sh.red[ww][hh]);
+            const float tmax = tmx[hh];
             bool k = hh < G;
             if (kScreen && k) k = (l[hh] == 0.f) || (tmax >= m[hh] + __log2f(l[hh]) + p.thr2);
             mnew[hh] = m[hh];
@@ -349,9 +390,11 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, 1)
           if (p.tile_mask && tid < G)
             p.tile_mask[(static_cast<size_t>(b) * p.H + g * G + tid) * p.T + t] =
                 (keep >> tid) & 1u;
+          ps_prev[0] = 0.f;
+          ps_prev[1] = 0.f;
           if (keep) {
-            // P_t for retained heads (zero for the others) and its row sums
-            float ps[2] = {0.f, 0.f};
+            // P_t for retained heads (zero for the others) and this warp's row sums,
+            // which the next tile's barrier publishes
             const int h0 = (lane & 3) * 2;
 #pragma unroll
             for (int kb = 0; kb < KB; ++kb)
@@ -366,35 +409,32 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, 1)
                     const float mu = (mnew[hh] == NEG_INF) ? 0.f : mnew[hh];
                     pv = fast_exp2(sc[kb][r8 * 2 + c] - mu);
                   }
-                  ps[c] += pv;
+                  ps_prev[c] += pv;
                   if (hh < G) sh.P[slot][hh][key] = __float2bfloat16(pv);
                 }
               }
 #pragma unroll
             for (int o = 4; o < 32; o <<= 1) {
-              ps[0] += __shfl_xor_sync(0xffffffffu, ps[0], o);
-              ps[1] += __shfl_xor_sync(0xffffffffu, ps[1], o);
-            }
-            named_bar_sync(1, NT);  // everyone has read sh.red (maxima)
-            if (lane < 2) {
-              sh.red[warp][lane * 2] = ps[0];
-              sh.red[warp][lane * 2 + 1] = ps[1];
+              ps_prev[0] += __shfl_xor_sync(0xffffffffu, ps_prev[0], o);
+              ps_prev[1] += __shfl_xor_sync(0xffffffffu, ps_prev[1], o);
             }
             if (tid < 8) sh.alpha[slot][tid] = (tid < 4) ? alpha[tid] : 1.f;
-            named_bar_sync(1, NT);
-#pragma unroll
-            for (int hh = 0; hh < 4; ++hh) {
-              if ((keep >> hh) & 1u) {
-                float tsum = 0.f;
-#pragma unroll
-                for (int ww = 0; ww < CW; ++ww) tsum += sh.red[ww][hh];
-                l[hh] = l[hh] * alpha[hh] + tsum;
-                m[hh] = mnew[hh];
-              }
-            }
           }
-          named_bar_sync(1, NT);  // sh.red is reused by the next tile
+          pkeep = keep;
+#pragma unroll
+          for (int hh = 0; hh < 4; ++hh) { palpha[hh] = alpha[hh]; pmnew[hh] = mnew[hh]; }
+        } else if (n == nt) {
+          // close the unit's last tile; this barrier also orders its P and alpha before
+          // the P.V of the iterations that follow
+          const int rb = n & 1;
+          if (lane < 2) {
+            float* rs = reinterpret_cast<float*>(&sh.rsum[rb][warp]);
+            rs[lane * 2] = ps_prev[0];
+            rs[lane * 2 + 1] = ps_prev[1];
+          }
+          named_bar_sync(1, NT);
           if (*ast.flag) { ok = false; break; }
+          close_tile(rb);
         }
         // P.V of the tile decided kLag iterations ago
         if (n >= kLag) {
