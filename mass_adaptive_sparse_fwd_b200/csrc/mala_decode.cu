@@ -42,7 +42,10 @@ int sm_count();
 namespace {
 
 constexpr int kLag = 2;        // tiles between a decision and its P.V
-constexpr int kPR = kLag + 1;  // P / decision ring depth
+// P / decision ring depth: P of tile n is written before tile n's barrier, while a slower
+// warp may still be in the P.V of tile n - kLag - 1 (before that barrier); slot n was last
+// read by the P.V of tile n - kLag - 2, which every warp finished before barrier n - 1
+constexpr int kPR = kLag + 2;
 
 template <int D>
 struct DecCfg {
@@ -78,15 +81,15 @@ struct DecShared {
   uint64_t k_full[6], k_empty[6], v_full[6], v_empty[6];
   uint64_t dec_full[kPR], dec_empty[kPR];
   __nv_bfloat16 qs[8][128];           // query rows of the group, heads >= G are zero
-  // P_t, rows = heads (>= G zero); rows padded by 8 keys so that the P.V fragment
-  // loads (8 heads x 4 key pairs per warp) fall on 32 distinct banks
-  __nv_bfloat16 P[kPR][8][kTile + 8];
-  float alpha[kPR][8];                // rescale of O at tile t, per head
+  // P_t in fp32, rows = heads (>= G zero), each warp's keys relative to that warp's own
+  // maximum; rows padded by 8 keys (bank spread of the P.V fragment loads)
+  alignas(16) float P[kPR][8][kTile + 8];
+  float beta[kPR][8][4];              // [key segment][head]: 2^(segment max - new max)
+  float alpha[kPR][4];                // rescale of O at tile t, per head
   uint32_t keep[kPR];                 // bit h: head h retained tile t
-  // per-warp partial tile maxima of tile n and row sums of tile n - 1 (heads 0..3),
-  // double-buffered by the parity of n
-  float4 rmax[2][8];
-  float4 rsum[2][8];
+  // per-warp tile maxima and row sums (heads 0..3), double-buffered by tile parity
+  float rmax[2][8][4];
+  float rsum[2][8][4];
   uint32_t last_flag;
   uint32_t abort_flag;
 };
@@ -239,8 +242,12 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, 1)
     // zero the padded heads of P once (rows >= G are never written again)
     for (int i = tid; i < kPR * 8 * (kTile + 8); i += NT) {
       const int row = (i / (kTile + 8)) % 8;
-      if (row >= G) (&sh.P[0][0][0])[i] = __float2bfloat16(0.f);
+      if (row >= G) (&sh.P[0][0][0])[i] = 0.f;
     }
+    // decision lanes: lane L of every consumer warp handles key segment (warp) dw and
+    // head dh; the per-head state m, l lives in the lanes of that head (replicated over
+    // the 8 segment lanes, and over warps: every warp takes the same decisions)
+    const int dw = lane & 7, dh = lane >> 3;
     for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
       int b, g, s, t_lo, t_hi;
       unit_coords(p, u, b, g, s, t_lo, t_hi);
@@ -260,32 +267,7 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, 1)
         qb[ks][0] = *reinterpret_cast<const uint32_t*>(&sh.qs[hh][c0]);
         qb[ks][1] = *reinterpret_cast<const uint32_t*>(&sh.qs[hh][c0 + 8]);
       }
-      // per-head running state (replicated in every consumer thread).  The normaliser
-      // update of tile n (l = l alpha + row sum, m = mnew) is applied after the next
-      // barrier, which publishes the row sums; the test of tile n + 1 comes after it.
-      float m[4], l[4], palpha[4], pmnew[4];
-      float ps_prev[2] = {0.f, 0.f};  // this warp's row sums of the last decided tile
-      uint32_t pkeep = 0;
-#pragma unroll
-      for (int hh = 0; hh < 4; ++hh) {
-        m[hh] = NEG_INF; l[hh] = 0.f; palpha[hh] = 1.f; pmnew[hh] = NEG_INF;
-      }
-      auto close_tile = [&](int rb) {
-        if (!pkeep) return;
-        float4 ts4 = sh.rsum[rb][0];
-#pragma unroll
-        for (int ww = 1; ww < CW; ++ww) {
-          const float4 v4 = sh.rsum[rb][ww];
-          ts4.x += v4.x; ts4.y += v4.y; ts4.z += v4.z; ts4.w += v4.w;
-        }
-        const float tsum[4] = {ts4.x, ts4.y, ts4.z, ts4.w};
-#pragma unroll
-        for (int hh = 0; hh < 4; ++hh)
-          if ((pkeep >> hh) & 1u) {
-            l[hh] = l[hh] * palpha[hh] + tsum[hh];
-            m[hh] = pmnew[hh];
-          }
-      };
+      float m_h = NEG_INF, l_h = 0.f;  // running state of head dh (online, log2 units)
       // O^T accumulators: warp owns head-dim rows [16 MB w, 16 MB (w+1))
       float acc[MB][4];
 #pragma unroll
@@ -301,7 +283,7 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, 1)
           // A failed wait only raises the abort flag; the consumers leave the loop
           // together, right after their next named barrier.
           const bool got = mbar_wait_warp(&sh.k_full[kst], (kc / NK) & 1, ast, 10);
-          // scores of this warp's 32 keys x 8 (padded) heads
+          // scores of this warp's keys x 8 (padded) heads
           float sc[KB][4];
 #pragma unroll
           for (int kb = 0; kb < KB; ++kb) {
@@ -322,7 +304,10 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, 1)
           __syncwarp();
           if (lane == 0) mbar_arrive(&sh.k_empty[kst]);
           ++kc;
-          // scale into log2 units, mask keys past the end, per-head tile maxima
+          // log2-domain scores (keys past the end masked), this warp's maxima and
+          // P relative to them, written before the decision: thread columns are heads
+          // h0 and h0 + 1, rows are keys
+          const int h0 = (lane & 3) * 2;
           float mx[2] = {NEG_INF, NEG_INF};
 #pragma unroll
           for (int kb = 0; kb < KB; ++kb)
@@ -339,45 +324,68 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, 1)
             mx[0] = fmaxf(mx[0], __shfl_xor_sync(0xffffffffu, mx[0], o));
             mx[1] = fmaxf(mx[1], __shfl_xor_sync(0xffffffffu, mx[1], o));
           }
-          // the tile's only barrier: this tile's per-warp maxima travel together with
-          // the previous tile's per-warp row sums
+          float ps[2] = {0.f, 0.f};
+#pragma unroll
+          for (int kb = 0; kb < KB; ++kb)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int c = e & 1, hh = h0 + c;
+              const float mu = (mx[c] == NEG_INF) ? 0.f : mx[c];
+              const float pv = fast_exp2(sc[kb][e] - mu);
+              ps[c] += pv;
+              if (hh < G)
+                sh.P[slot][hh][warp * (16 * KB) + kb * 16 + (lane >> 2) + (e >> 1) * 8] = pv;
+            }
+#pragma unroll
+          for (int o = 4; o < 32; o <<= 1) {
+            ps[0] += __shfl_xor_sync(0xffffffffu, ps[0], o);
+            ps[1] += __shfl_xor_sync(0xffffffffu, ps[1], o);
+          }
           const int rb = n & 1;
           if (lane < 2) {  // lanes 0, 1 hold heads 0-1 and 2-3
-            float* rm = reinterpret_cast<float*>(&sh.rmax[rb][warp]);
-            float* rs = reinterpret_cast<float*>(&sh.rsum[rb][warp]);
-            rm[lane * 2] = mx[0];
-            rm[lane * 2 + 1] = mx[1];
-            rs[lane * 2] = ps_prev[0];
-            rs[lane * 2 + 1] = ps_prev[1];
+            sh.rmax[rb][warp][lane * 2] = mx[0];
+            sh.rmax[rb][warp][lane * 2 + 1] = mx[1];
+            sh.rsum[rb][warp][lane * 2] = ps[0];
+            sh.rsum[rb][warp][lane * 2 + 1] = ps[1];
           }
+          // the tile's only barrier; it also orders the P, beta and alpha of older
+          // tiles before their P.V below
           named_bar_sync(1, NT);
           if (*ast.flag) { ok = false; break; }
-          if (n > 0) close_tile(rb);
-          // retention test per head (Eq. 3 with L_0 = N_k), identical in every thread
-          float4 tm4 = sh.rmax[rb][0];
-#pragma unroll
-          for (int ww = 1; ww < CW; ++ww) {
-            const float4 v4 = sh.rmax[rb][ww];
-            tm4.x = fmaxf(tm4.x, v4.x); tm4.y = fmaxf(tm4.y, v4.y);
-            tm4.z = fmaxf(tm4.z, v4.z); tm4.w = fmaxf(tm4.w, v4.w);
-          }
-          const float tmx[4] = {tm4.x, tm4.y, tm4.z, tm4.w};
-          uint32_t keep = 0;
-          float mnew[4], alpha[4];
-#pragma unroll
-          for (int hh = 0; hh < 4; ++hh) {
-            const float tmax = tmx[hh];
-            bool k = hh < G;
-            if (kScreen && k) k = (l[hh] == 0.f) || (tmax >= m[hh] + __log2f(l[hh]) + p.thr2);
-            mnew[hh] = m[hh];
-            alpha[hh] = 1.f;
-            if (k) {
-              keep |= 1u << hh;
-              if (tmax > m[hh] + 8.0f) {
-                mnew[hh] = tmax;
-                alpha[hh] = fast_exp2(m[hh] - tmax);  // 0 on the first retained tile
-              }
+          // retention test of head dh (Eq. 3 with L_0 = N_k) on the tile maximum, and
+          // the normaliser update l = l alpha + sum_w rowsum_w 2^(max_w - m_new)
+          const float mv = (dw < CW) ? sh.rmax[rb][dw][dh] : NEG_INF;
+          const float sv = (dw < CW) ? sh.rsum[rb][dw][dh] : 0.f;
+          float tmax = mv;
+          tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 1));
+          tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 2));
+          tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 4));
+          bool k = dh < G;
+          if (kScreen && k) k = (l_h == 0.f) || (tmax >= m_h + __log2f(l_h) + p.thr2);
+          float mnew = m_h, alpha = 1.f, beta = 0.f;
+          if (k) {
+            if (tmax > m_h + 8.0f) {
+              mnew = tmax;
+              alpha = fast_exp2(m_h - tmax);  // 0 on the first retained tile
             }
+            beta = fast_exp2(mv - mnew);      // 0 for a segment with no valid key
+          }
+          float sum = sv * beta;
+          sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+          sum += __shfl_xor_sync(0xffffffffu, sum, 2);
+          sum += __shfl_xor_sync(0xffffffffu, sum, 4);
+          if (k) {
+            l_h = l_h * alpha + sum;
+            m_h = mnew;
+          }
+          const uint32_t bal = __ballot_sync(0xffffffffu, k);
+          const uint32_t keep = (bal & 1u) | ((bal >> 7) & 2u) | ((bal >> 14) & 4u) |
+                                ((bal >> 21) & 8u);
+          if (warp == 0) {
+            if (dw < CW) sh.beta[slot][dw][dh] = beta;
+            if (dw == 0) sh.alpha[slot][dh] = alpha;
+            if (p.tile_mask && dw == 0 && dh < G)
+              p.tile_mask[(static_cast<size_t>(b) * p.H + g * G + dh) * p.T + t] = k ? 1 : 0;
           }
           // hand the decision to the V producer (ring slot must be free)
           if (tid == 0) {
@@ -387,54 +395,10 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, 1)
             sh.keep[slot] = keep;
             if (free_slot) mbar_arrive(&sh.dec_full[slot]);
           }
-          if (p.tile_mask && tid < G)
-            p.tile_mask[(static_cast<size_t>(b) * p.H + g * G + tid) * p.T + t] =
-                (keep >> tid) & 1u;
-          ps_prev[0] = 0.f;
-          ps_prev[1] = 0.f;
-          if (keep) {
-            // P_t for retained heads (zero for the others) and this warp's row sums,
-            // which the next tile's barrier publishes
-            const int h0 = (lane & 3) * 2;
-#pragma unroll
-            for (int kb = 0; kb < KB; ++kb)
-#pragma unroll
-              for (int r8 = 0; r8 < 2; ++r8) {
-                const int key = warp * (16 * KB) + kb * 16 + (lane >> 2) + r8 * 8;
-#pragma unroll
-                for (int c = 0; c < 2; ++c) {
-                  const int hh = h0 + c;
-                  float pv = 0.f;
-                  if (hh < 4 && ((keep >> hh) & 1u)) {
-                    const float mu = (mnew[hh] == NEG_INF) ? 0.f : mnew[hh];
-                    pv = fast_exp2(sc[kb][r8 * 2 + c] - mu);
-                  }
-                  ps_prev[c] += pv;
-                  if (hh < G) sh.P[slot][hh][key] = __float2bfloat16(pv);
-                }
-              }
-#pragma unroll
-            for (int o = 4; o < 32; o <<= 1) {
-              ps_prev[0] += __shfl_xor_sync(0xffffffffu, ps_prev[0], o);
-              ps_prev[1] += __shfl_xor_sync(0xffffffffu, ps_prev[1], o);
-            }
-            if (tid < 8) sh.alpha[slot][tid] = (tid < 4) ? alpha[tid] : 1.f;
-          }
-          pkeep = keep;
-#pragma unroll
-          for (int hh = 0; hh < 4; ++hh) { palpha[hh] = alpha[hh]; pmnew[hh] = mnew[hh]; }
         } else if (n == nt) {
-          // close the unit's last tile; this barrier also orders its P and alpha before
-          // the P.V of the iterations that follow
-          const int rb = n & 1;
-          if (lane < 2) {
-            float* rs = reinterpret_cast<float*>(&sh.rsum[rb][warp]);
-            rs[lane * 2] = ps_prev[0];
-            rs[lane * 2 + 1] = ps_prev[1];
-          }
+          // orders the last tile's P, beta, alpha and keep before the P.V that follow
           named_bar_sync(1, NT);
           if (*ast.flag) { ok = false; break; }
-          close_tile(rb);
         }
         // P.V of the tile decided kLag iterations ago
         if (n >= kLag) {
@@ -453,11 +417,16 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, 1)
               acc[mb][0] *= a0; acc[mb][1] *= a1; acc[mb][2] *= a0; acc[mb][3] *= a1;
             }
             const uint32_t vbase = sVa + vst * C::TILE_BYTES;
+            const int hh = lane >> 2;  // B-fragment column (head) of this thread
 #pragma unroll
             for (int ks = 0; ks < (vgot ? kTile / 16 : 0); ++ks) {
-              const int hh = lane >> 2, kk = ks * 16 + (lane & 3) * 2;
-              const uint32_t b0 = *reinterpret_cast<const uint32_t*>(&sh.P[slot2][hh][kk]);
-              const uint32_t b1 = *reinterpret_cast<const uint32_t*>(&sh.P[slot2][hh][kk + 8]);
+              // P of key segment ks / KB, scaled to the tile's new maximum
+              const float bt = (hh < 4) ? sh.beta[slot2][ks / KB][hh] : 0.f;
+              const int kk = ks * 16 + (lane & 3) * 2;
+              const float2 p0 = *reinterpret_cast<const float2*>(&sh.P[slot2][hh][kk]);
+              const float2 p1 = *reinterpret_cast<const float2*>(&sh.P[slot2][hh][kk + 8]);
+              const uint32_t b0 = pack_bf16(p0.x * bt, p0.y * bt);
+              const uint32_t b1 = pack_bf16(p1.x * bt, p1.y * bt);
 #pragma unroll
               for (int mb = 0; mb < MB; ++mb) {
                 const int d0 = warp * (16 * MB) + mb * 16;
@@ -472,8 +441,6 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(&sh.v_empty[vst]);
             ++vc;
-          } else {
-            // nothing retained: O keeps its scale (alpha = 1 for every head)
           }
         }
       }
@@ -481,24 +448,25 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, 1)
       n_glob += nt;
       named_bar_sync(1, NT);
       if (*ast.flag) { ok = false; break; }
-      // this split's normalised output o_s = acc / l and z_s = (m + log2 l) ln 2
+      // this split's normalised output o_s = acc / l and z_s = (m + log2 l) ln 2; the
+      // state of head h sits in lanes 8h .. 8h+7
       {
         const int h0 = (lane & 3) * 2;
+        const float la = __shfl_sync(0xffffffffu, l_h, (h0 & 3) * 8);
+        const float lb = __shfl_sync(0xffffffffu, l_h, ((h0 + 1) & 3) * 8);
 #pragma unroll
         for (int mb = 0; mb < MB; ++mb)
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int hh = h0 + (e & 1);
             const int dd = warp * (16 * MB) + mb * 16 + (lane >> 2) + (e >> 1) * 8;
-            if (hh < G) {
-              const float lv = (hh == 0) ? l[0] : (hh == 1) ? l[1] : (hh == 2) ? l[2] : l[3];
+            if (hh < G)
               p.part_o[((static_cast<size_t>(b) * p.H + g * G + hh) * p.S + s) * D + dd] =
-                  acc[mb][e] / lv;
-            }
+                  acc[mb][e] / ((e & 1) ? lb : la);
           }
-        if (tid < G)
-          p.part_z[(static_cast<size_t>(b) * p.H + g * G + tid) * p.S + s] =
-              (m[tid] + __log2f(l[tid])) * kLn2;
+        if (warp == 0 && dw == 0 && dh < G)
+          p.part_z[(static_cast<size_t>(b) * p.H + g * G + dh) * p.S + s] =
+              (m_h + __log2f(l_h)) * kLn2;
       }
       // last CTA of this (b, g) merges the splits
       named_bar_sync(1, NT);
