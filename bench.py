@@ -37,6 +37,7 @@ from mass_adaptive_sparse_fwd_b200 import synth  # noqa: E402
 METRIC = "MALA fwd+bwd ms and TFLOPS at 32K, decode µs at 128K; % of bf16 tensor peak"
 TRAIN = "sinkband32k"  # --train sinkband128k times the 128K one-GPU training shape instead
 SKIP_TRAIN = "prevtok32k"  # concentrated states for the skip-regime block
+SKIP_DECODE = "heavy128k"  # KV cache with a heavy hitter in every 8th key tile
 DECODE = "decode128k"
 TAU = 1.0
 KERNELS_PER_STEP = 5  # fwd 1, bwd 3 (D preprocess, main, dQ convert), decode 1
@@ -496,6 +497,60 @@ def run_mala(args, dist: Dist):
                 "work_ratio": {"fwd": sfl["fwd_exec"] / sfl0["fwd_exec"],
                                "bwd": sfl["bwd_exec"] / sfl0["bwd_exec"]}}
         del sQ, sK, sV, sdO, sO, sLSE, sdQ, sdK, sdV, swf, swb
+
+        # decode on a cache whose every split holds dominant keys: the tiles between
+        # them, and their V loads, are skipped
+        wh = rank_workload(synth.WORKLOADS[SKIP_DECODE], dist.rank)
+        loc = synth.make_decode(wh)
+        hq, hK, hV = (bf(loc[k]) for k in ("q", "K", "V"))
+        del loc
+        hO = torch.empty_like(hq)
+        hL = torch.empty((wh.B, wh.H), dtype=torch.float32, device=dev)
+        hS = mala.decode_num_splits(wh.B, wh.H, wh.H_kv, wh.L)
+        hws = mala.alloc_workspace(
+            mala.decode_workspace_bytes(wh.B, wh.H, wh.H_kv, wh.L, wh.d, 0, hS), dev)
+
+        def hdec(tau, mask=None):
+            mala.mala_decode(hq, hK, hV, wh.scale, tau, num_splits=hS, O=hO, LSE=hL,
+                             workspace=hws, tile_mask=mask)
+
+        def dtime(tau):
+            for _ in range(args.warmup):
+                hdec(tau)
+            torch.cuda.synchronize(dev)
+            dist.barrier()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(args.steps):
+                hdec(tau)
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            dist.barrier()
+            err = mala.read_device_error(hws)
+            if err:
+                raise RuntimeError(f"device error word 0x{err:x}")
+            return dist.max(e0.elapsed_time(e1) / args.steps * 1e3, device=dev)
+
+        hd1 = dtime(TAU)
+        hd0 = dtime(0.0)
+        hT = mala.n_tiles(wh.L)
+        hmask = torch.zeros((wh.B, wh.H, hT), dtype=torch.uint8, device=dev)
+        hdec(TAU, hmask)
+        torch.cuda.synchronize(dev)
+        hG = wh.H // wh.H_kv
+        hv = int(hmask.view(wh.B, wh.H_kv, hG, -1).amax(dim=2).sum())
+        hb1 = decode_bytes(wh, hv, hS)
+        hb0 = decode_bytes(wh, wh.B * wh.H_kv * hT, hS)
+        skip["decode"] = {
+            "workload": f"{SKIP_DECODE} (B={wh.B},H={wh.H},H_kv={wh.H_kv},N_k={wh.L},d={wh.d}; "
+                        "a heavy hitter shared by each KV group in every 8th key tile)",
+            "splits": hS,
+            "retained": {"tiles": float(hmask.float().mean()),
+                         "v_tiles": hv / (wh.B * wh.H_kv * hT)},
+            "tau1_us": hd1, "tau0_us": hd0, "speedup_vs_tau0": hd0 / hd1,
+            "bytes_ratio": hb1 / hb0,
+            "tau1_gbs": hb1 / (hd1 * 1e-6) / 1e9, "tau0_gbs": hb0 / (hd0 * 1e-6) / 1e9}
+        del hq, hK, hV, hO, hL, hws
 
     cpu = None
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:

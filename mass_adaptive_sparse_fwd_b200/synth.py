@@ -24,6 +24,9 @@ available; these synthetic distributions stand in for them):
 * ``decode128k``  B=4, H=32, H_kv=8, N_k=131072, d=128, bf16; K, V, q ~ N(0, 1); per
                   (b, KV head) 16 distinct random positions get a planted key
                   3.0 * sqrt(d) * q_h / |q_h| + N(0, 1), h cycling over the group's heads
+* ``heavy128k``   decode128k's shape, K, V, q ~ N(0, 1), with one heavy hitter per
+                  (b, KV head) at key 64 of every 8th tile (tiles 7, 15, ...):
+                  28 * sum_h q_h / |q_h| + 0.1 N(0, 1) over the group's heads
 * ``sinkband128k`` B=1, H=8, H_kv=1, L=131072, d=128, bf16; sink + band states as
                   ``sinkband32k`` (one rank of an 8-way head-sharded 64/8-head model)
 * ``prevtok32k``  B=1, H=32, H_kv=8, L=32768, d=128, bf16; concentrated "previous-token"
@@ -74,6 +77,10 @@ WORKLOADS = {
     "sinkband32k": Workload("sinkband32k", 1, 32, 8, 32768, 128, "bf16", "sink_band", 3),
     "decode128k": Workload("decode128k", 4, 32, 8, 131072, 128, "bf16", "planted", 4,
                            decode=True),
+    # decode with a heavy hitter every 8th key tile: every split holds dominant keys, so
+    # the tiles between them (and their V) are skipped
+    "heavy128k": Workload("heavy128k", 4, 32, 8, 131072, 128, "bf16", "heavy", 7,
+                          decode=True),
     # 128K-token training on one GPU: the per-rank shape of a 64-query-head / 8-KV-head
     # model under 8-way head sharding, with the sink + band states of sinkband32k
     "sinkband128k": Workload("sinkband128k", 1, 8, 1, 131072, 128, "bf16", "sink_band", 5),
@@ -220,15 +227,30 @@ def make_decode(w: Workload, Nk: int | None = None, B: int | None = None) -> dic
     K = normal(w.seed, _K, (B, Nk, Hkv, d), w.dtype)
     V = normal(w.seed, _V, (B, Nk, Hkv, d), w.dtype)
     rng = _rng(w.seed, _PLANT)
-    n_plant = min(16, Nk)
-    for b in range(B):
-        for g in range(Hkv):
-            pos = rng.choice(Nk, size=n_plant, replace=False)
-            for r, p in enumerate(pos):
-                h = g * G + (r % G)
-                qh = q[b, h].astype(np.float64)
-                key = 3.0 * math.sqrt(d) * qh / np.linalg.norm(qh) + rng.standard_normal(d)
-                K[b, p, g] = _round(key.astype(np.float32), w.dtype)
+    if w.structure == "planted":
+        n_plant = min(16, Nk)
+        for b in range(B):
+            for g in range(Hkv):
+                pos = rng.choice(Nk, size=n_plant, replace=False)
+                for r, p in enumerate(pos):
+                    h = g * G + (r % G)
+                    qh = q[b, h].astype(np.float64)
+                    key = 3.0 * math.sqrt(d) * qh / np.linalg.norm(qh) + rng.standard_normal(d)
+                    K[b, p, g] = _round(key.astype(np.float32), w.dtype)
+    elif w.structure == "heavy":
+        # one heavy hitter shared by the group in every 8th key tile (key 64 of tiles
+        # 7, 15, 23, ...): k = 28 u + 0.1 N(0, 1), u = the sum of the group's unit query
+        # directions, so each head scores it near 28 (|q_h| ~ sqrt(d), nearly orthogonal
+        # query directions) against ~N(0, 1) for the other keys
+        for b in range(B):
+            for g in range(Hkv):
+                qg = q[b, g * G:(g + 1) * G].astype(np.float64)
+                u = (qg / np.linalg.norm(qg, axis=-1, keepdims=True)).sum(axis=0)
+                for p in range(7 * 128 + 64, Nk, 8 * 128):
+                    key = 28.0 * u + 0.1 * rng.standard_normal(d)
+                    K[b, p, g] = _round(key.astype(np.float32), w.dtype)
+    else:
+        raise ValueError(w.structure)
     return {"q": q, "K": K, "V": V}
 
 

@@ -94,3 +94,22 @@ def test_decode_fp32(orc, mala, tau):
     w = synth.Workload("fp32_decode", 2, 4, 2, 700, 64, "fp32", "planted", 23, decode=True)
     inp = synth.make_decode(w)
     check_decode(orc, mala, inp, w.scale, tau, 2, dtype="fp32")
+
+
+@pytest.mark.parametrize("S", [2, 5])
+def test_decode_heavy_small(orc, mala, S):
+    """Heavy hitters in every split: most tiles and most V loads are skipped."""
+    w = synth.Workload("adhoc_heavy", 2, 8, 2, 8192, 128, "bf16", "heavy", 24, decode=True)
+    inp = synth.make_decode(w)
+    mask = check_decode(orc, mala, inp, w.scale, 1.0, S)
+    group = mask.reshape(w.B, w.H_kv, w.H // w.H_kv, -1).max(axis=2)
+    assert group.mean() < 0.5
+
+
+def test_heavy128k_full(orc, mala):
+    w = synth.WORKLOADS["heavy128k"]
+    inp = synth.make_decode(w)
+    S = mala.decode_num_splits(w.B, w.H, w.H_kv, w.L)
+    mask = check_decode(orc, mala, inp, w.scale, 1.0, S)
+    group = mask.reshape(w.B, w.H_kv, w.H // w.H_kv, -1).max(axis=2)
+    assert group.mean() < 0.35
