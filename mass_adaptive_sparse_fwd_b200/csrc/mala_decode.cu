@@ -280,6 +280,7 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, 1)
           const int t = t_hi - 1 - n;
           const uint32_t slot = (n_glob + n) % kPR;
           const int kst = kc % NK;
+          const float cut = m_h + __log2f(l_h) + p.thr2;
           // A failed wait only raises the abort flag; the consumers leave the loop
           // together, right after their next named barrier.
           const bool got = mbar_wait_warp(&sh.k_full[kst], (kc / NK) & 1, ast, 10);
@@ -361,32 +362,34 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, 1)
           tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 2));
           tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 4));
           bool k = dh < G;
-          if (kScreen && k) k = (l_h == 0.f) || (tmax >= m_h + __log2f(l_h) + p.thr2);
-          float mnew = m_h, alpha = 1.f, beta = 0.f;
-          if (k) {
-            if (tmax > m_h + 8.0f) {
-              mnew = tmax;
-              alpha = fast_exp2(m_h - tmax);  // 0 on the first retained tile
-            }
-            beta = fast_exp2(mv - mnew);      // 0 for a segment with no valid key
-          }
-          float sum = sv * beta;
-          sum += __shfl_xor_sync(0xffffffffu, sum, 1);
-          sum += __shfl_xor_sync(0xffffffffu, sum, 2);
-          sum += __shfl_xor_sync(0xffffffffu, sum, 4);
-          if (k) {
-            l_h = l_h * alpha + sum;
-            m_h = mnew;
-          }
+          if (kScreen && k) k = (l_h == 0.f) || (tmax >= cut);
           const uint32_t bal = __ballot_sync(0xffffffffu, k);
           const uint32_t keep = (bal & 1u) | ((bal >> 7) & 2u) | ((bal >> 14) & 4u) |
                                 ((bal >> 21) & 8u);
-          if (warp == 0) {
-            if (dw < CW) sh.beta[slot][dw][dh] = beta;
-            if (dw == 0) sh.alpha[slot][dh] = alpha;
-            if (p.tile_mask && dw == 0 && dh < G)
-              p.tile_mask[(static_cast<size_t>(b) * p.H + g * G + dh) * p.T + t] = k ? 1 : 0;
+          if (bal) {  // warp-uniform: some head keeps the tile
+            float mnew = m_h, alpha = 1.f, beta = 0.f;
+            if (k) {
+              if (tmax > m_h + 8.0f) {
+                mnew = tmax;
+                alpha = fast_exp2(m_h - tmax);  // 0 on the first retained tile
+              }
+              beta = fast_exp2(mv - mnew);      // 0 for a segment with no valid key
+            }
+            float sum = sv * beta;
+            sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+            sum += __shfl_xor_sync(0xffffffffu, sum, 2);
+            sum += __shfl_xor_sync(0xffffffffu, sum, 4);
+            if (k) {
+              l_h = l_h * alpha + sum;
+              m_h = mnew;
+            }
+            if (warp == 0) {
+              if (dw < CW) sh.beta[slot][dw][dh] = beta;
+              if (dw == 0) sh.alpha[slot][dh] = alpha;
+            }
           }
+          if (warp == 0 && p.tile_mask && dw == 0 && dh < G)
+            p.tile_mask[(static_cast<size_t>(b) * p.H + g * G + dh) * p.T + t] = k ? 1 : 0;
           // hand the decision to the V producer (ring slot must be free)
           if (tid == 0) {
             bool free_slot = true;
