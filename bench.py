@@ -602,6 +602,32 @@ def run_mala(args, dist: Dist):
         print(json.dumps(line), flush=True)
 
 
+def profile_case(case: str):
+    """Two rounds (warm-up, then the one to capture) of the three main kernels on
+    mid-size inputs for an ncu capture: a few GB on the device, inputs larger than L2.
+    case "headline": sink + band states, B=1, H=32, H_kv=8, L=8192 and the planted
+    decode cache at N_k=32768; case "skip": previous-token states at L=8192 and the
+    heavy-hitter cache at N_k=32768.  tau = 1."""
+    from mass_adaptive_sparse_fwd_b200 import mala
+
+    train, dec = (("sinkband32k", "decode128k") if case == "headline"
+                  else ("prevtok32k", "heavy128k"))
+    wt, wd = synth.WORKLOADS[train], synth.WORKLOADS[dec]
+    tr = synth.make_training(wt, L=8192)
+    dc = synth.make_decode(wd, Nk=32768)
+    bf = lambda x: torch.from_numpy(x).cuda().to(torch.bfloat16)
+    Q, K, V, dO = (bf(tr[k]) for k in ("Q", "K", "V", "dO"))
+    q, Kc, Vc = (bf(dc[k]) for k in ("q", "K", "V"))
+    for _ in range(2):
+        O, LSE = mala.mala_fwd(Q, K, V, wt.scale, TAU)
+        dQ, dK, dV = mala.mala_bwd(Q, K, V, O, LSE, dO, wt.scale, TAU)
+        Od, _ = mala.mala_decode(q, Kc, Vc, wd.scale, TAU)
+        torch.cuda.synchronize()
+    print(json.dumps({"profile_case": case, "O": float(O.float().abs().mean()),
+                      "dQ": float(dQ.float().abs().mean()),
+                      "O_decode": float(Od.float().abs().mean())}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -613,7 +639,12 @@ def main():
     ap.add_argument("--no-skip-regime", action="store_true")
     ap.add_argument("--train", default=TRAIN, choices=("sinkband32k", "sinkband128k"),
                     help="training workload of the step (default: the 32K headline shape)")
+    ap.add_argument("--profile-case", choices=("headline", "skip"),
+                    help="run the kernels once on a mid-size case for an ncu capture and exit")
     args = ap.parse_args()
+    if args.profile_case:
+        profile_case(args.profile_case)
+        return
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     dist = Dist()
