@@ -579,6 +579,10 @@ def run_mala(args, dist: Dist):
             "retained": {"fwd_tiles": fret, "bwd_tiles": bret, "decode_tiles": dret,
                          "decode_v_tiles": vtiles / (wd.B * wd.H_kv * mala.n_tiles(wd.L)),
                          "fwd_slots_per_query": fret * (L + 128) / 2.0},
+            # exponentials evaluated (one per score of a retained tile; Eq. (13)/(16) counts)
+            "exp_count": {"fwd": 128 * 128 * round(fret * fl["legal_tiles"]),
+                          "bwd": 128 * 128 * round(bret * fl["legal_tiles"]),
+                          "dense": 128 * 128 * fl["legal_tiles"]},
             "decode_gbs": dec_gbs,
             "dense_tau0": {"fwd_ms": res0["fwd_ms"], "bwd_ms": res0["bwd_ms"],
                            "fwd_bwd_ms": dense_fb, "decode_us": res0["decode_ms"] * 1e3,

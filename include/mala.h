@@ -128,6 +128,26 @@ mala_status mala_decode_noalloc(const void* q, const void* Kc, const void* Vc, v
                                 float scale, float tau, int num_splits, unsigned flags,
                                 uint8_t* tile_mask, void* stream);
 
+/*
+ * mala_get_stats - work statistics of the last call that ran on `workspace`.
+ * The attention page reports the retained fraction of post-score work (§3); these counters
+ * give it without a tile_mask buffer.  Every call that receives a caller workspace zeroes
+ * them first and its kernels add to them (the fp32 forward, which needs no workspace,
+ * fills them when one is passed anyway).  Synchronises `stream`.
+ *   Forward / backward: legal_tiles = causal tiles tested, one per (b, h, i, j);
+ *   retained_tiles = tiles whose post-score work ran; v_tiles_loaded = 0.
+ *   Decode: legal_tiles = (b, h, key tile) pairs tested; retained_tiles = pairs retained;
+ *   v_tiles_loaded = V tiles fetched (one per (b, KV head, tile) that some head of the
+ *   group retains; per (b, h) on the fp32 path).
+ * Calls made with workspace == NULL, and mala_decode_noalloc, keep no statistics.
+ */
+typedef struct {
+  uint64_t legal_tiles;
+  uint64_t retained_tiles;
+  uint64_t v_tiles_loaded;
+} mala_stats;
+mala_status mala_get_stats(const void* workspace, void* stream, mala_stats* out);
+
 /* Workspace sizes (bytes) for the calls above; 0 on invalid arguments. */
 size_t mala_fwd_workspace_bytes(int B, int H, int H_kv, int L, int d, int dtype);
 size_t mala_bwd_workspace_bytes(int B, int H, int H_kv, int L, int d, int dtype);

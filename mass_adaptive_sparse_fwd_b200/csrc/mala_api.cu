@@ -29,7 +29,7 @@ size_t decode_workspace_bytes(int B, int H, int Hkv, int Nk, int d, int dtype, i
 int decode_auto_splits(int B, int Hkv, int Nk);
 mala_status fp32_fwd(const float* Q, const float* K, const float* V, float* O, float* LSE, int B,
                      int H, int Hkv, int L, int d, float scale, float tau, bool screen,
-                     uint8_t* tile_mask, cudaStream_t stream);
+                     uint8_t* ws, uint8_t* tile_mask, cudaStream_t stream);
 
 // ---------------------------------------------------------------------------- shared host helpers
 
@@ -149,6 +149,20 @@ mala_status mala_read_device_error(const void* workspace, void* stream, uint32_t
   return MALA_OK;
 }
 
+mala_status mala_get_stats(const void* workspace, void* stream, mala_stats* out) {
+  if (!workspace || !out) return MALA_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  unsigned long long v[3] = {0, 0, 0};
+  if (cudaMemcpyAsync(v, static_cast<const uint8_t*>(workspace) + kStatsOffset, sizeof(v),
+                      cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return MALA_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return MALA_ERR_CUDA;
+  out->legal_tiles = v[0];
+  out->retained_tiles = v[1];
+  out->v_tiles_loaded = v[2];
+  return MALA_OK;
+}
+
 size_t mala_fwd_workspace_bytes(int B, int H, int H_kv, int L, int d, int dtype) {
   if (!common_args_ok(B, H, H_kv, L, d, dtype, 1.f, 0.f)) return 0;
   return kWorkspaceHeader;
@@ -167,9 +181,19 @@ mala_status mala_fwd(const void* Q, const void* K, const void* V, void* O, float
   const int T = (L + kTile - 1) / kTile;
   if (dtype == MALA_FP32) {
     if (d > 128) return MALA_ERR_UNSUPPORTED;
+    // this path needs no scratch; a caller's workspace only receives the call statistics
+    uint8_t* ws = nullptr;
+    if (workspace) {
+      if (workspace_bytes < kWorkspaceHeader) return MALA_ERR_WORKSPACE;
+      if (!aligned16(workspace)) return MALA_ERR_INVALID_ARG;
+      ws = static_cast<uint8_t*>(workspace);
+      if (cudaMemsetAsync(ws + kStatsOffset, 0, 3 * sizeof(unsigned long long), st) !=
+          cudaSuccess)
+        return MALA_ERR_CUDA;
+    }
     return fp32_fwd(static_cast<const float*>(Q), static_cast<const float*>(K),
                     static_cast<const float*>(V), static_cast<float*>(O), LSE, B, H, H_kv, L, d,
-                    scale, tau, screen, tile_mask, st);
+                    scale, tau, screen, ws, tile_mask, st);
   }
   if (d != 64 && d != 128) return MALA_ERR_UNSUPPORTED;
   if ((long long)B * L > (1ll << 31) || (long long)B * H * T > (1ll << 30))
@@ -183,7 +207,8 @@ mala_status mala_fwd(const void* Q, const void* K, const void* V, void* O, float
   const size_t need = mala_fwd_workspace_bytes(B, H, H_kv, L, d, dtype);
   return with_workspace(workspace, workspace_bytes, need, st, [&](uint8_t* ws) -> mala_status {
     uint32_t* hdr = reinterpret_cast<uint32_t*>(ws);
-    if (cudaMemsetAsync(hdr + kHdrSched0, 0, 3 * sizeof(uint32_t), st) != cudaSuccess)
+    if (cudaMemsetAsync(hdr + kHdrSched0, 0, 3 * sizeof(uint32_t), st) != cudaSuccess ||
+        cudaMemsetAsync(ws + kStatsOffset, 0, 3 * sizeof(unsigned long long), st) != cudaSuccess)
       return MALA_ERR_CUDA;
     FwdParams p;
     p.B = B; p.H = H; p.Hkv = H_kv; p.L = L; p.T = T; p.G = H / H_kv;
@@ -195,6 +220,7 @@ mala_status mala_fwd(const void* Q, const void* K, const void* V, void* O, float
     p.err = hdr + kHdrError;
     p.sched = hdr + kHdrSched0;
     p.budget_ns = wait_budget_ns();
+    p.stats = reinterpret_cast<unsigned long long*>(ws + kStatsOffset);
     const int grid = p.n_units < sm_count() ? p.n_units : sm_count();
     cudaError_t e = launch_fwd_bf16(tq, tk, tv, p, d, screen, grid, st);
     return e == cudaSuccess ? MALA_OK : MALA_ERR_CUDA;

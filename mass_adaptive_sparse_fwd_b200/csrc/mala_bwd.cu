@@ -77,6 +77,7 @@ struct BwdParams {
   __nv_bfloat16* dK;     // [B, L, Hkv, D]
   __nv_bfloat16* dV;
   uint8_t* tile_mask;    // [B, H, T, T] or null
+  unsigned long long* stats;  // call statistics (kStatsOffset) or null
   uint32_t* err;
   uint32_t* sched;
   uint64_t budget_ns;
@@ -362,6 +363,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
     const float NEG_INF = -INFINITY;
     uint32_t ntile = 0, nret = 0;
+    uint32_t st_legal = 0, st_ret = 0;  // call statistics (thread 128)
     bool ok = true;
     uint8_t* dsrow_base = sdS + wg * 16384;  // this warpgroup's 64-column atom
     for (uint32_t k = 0; ok; ++k) {
@@ -458,8 +460,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           named_bar_sync(1, 256);  // every S^T load done before P overwrites it
         }
         if (*ast.flag) { ok = false; break; }
-        if (p.tile_mask && tid == 128)
-          p.tile_mask[((static_cast<size_t>(w.b) * p.H + h) * p.T + i) * p.T + w.j] = keep ? 1 : 0;
+        if (tid == 128) {
+          ++st_legal;
+          st_ret += keep ? 1u : 0u;
+          if (p.tile_mask)
+            p.tile_mask[((static_cast<size_t>(w.b) * p.H + h) * p.T + i) * p.T + w.j] = keep ? 1 : 0;
+        }
         if (!keep) {
           if (tid == 128) sh.dec = 0;
           tc_fence_before();
@@ -529,6 +535,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         warp_arrive(&sh.ds_full);
       }
     }
+    if (tid == 128) stats_add(p.stats, st_legal, st_ret, 0);
   } else if (warp >= 12) {
     // ------------------------------------------------------------------ dQ drain + dK/dV epilogue
     const int wq = warp & 3;
@@ -744,6 +751,9 @@ mala_status bwd_dispatch(const void* Q, const void* K, const void* V, const void
                          unsigned flags, uint8_t* ws, uint8_t* tile_mask, uint64_t budget_ns,
                          cudaStream_t stream) {
   const bool screen = (tau > 0.f) || (flags & MALA_FLAG_ALWAYS_TEST);
+  if (cudaMemsetAsync(ws + kStatsOffset, 0, 3 * sizeof(unsigned long long), stream) !=
+      cudaSuccess)
+    return MALA_ERR_CUDA;
   if (dtype == MALA_FP32)
     return fp32_bwd(static_cast<const float*>(Q), static_cast<const float*>(K),
                     static_cast<const float*>(V), static_cast<const float*>(O), LSE,
@@ -784,6 +794,7 @@ mala_status bwd_dispatch(const void* Q, const void* K, const void* V, const void
   p.dK = static_cast<__nv_bfloat16*>(dK);
   p.dV = static_cast<__nv_bfloat16*>(dV);
   p.tile_mask = tile_mask;
+  p.stats = reinterpret_cast<unsigned long long*>(ws + kStatsOffset);
   p.err = hdr + kHdrError;
   p.sched = hdr + kHdrSched0;
   p.budget_ns = budget_ns;

@@ -19,6 +19,21 @@ enum HeaderWord : int {
   kHdrTickets = 16,   // decode merge tickets start here (not used by fwd/bwd)
 };
 
+// Call statistics in the workspace header: three uint64 counters at this byte offset,
+// zeroed at the start of every call (legal tiles tested, retained tiles, V tiles loaded
+// by decode).  Fwd / bwd count one per (b, h, i, j) tile; decode one per (b, h, t).
+constexpr int kStatsOffset = 128;
+
+#ifdef __CUDACC__
+__device__ __forceinline__ void stats_add(unsigned long long* stats, uint32_t legal,
+                                          uint32_t retained, uint32_t v_loaded) {
+  if (!stats) return;
+  if (legal) atomicAdd(stats + 0, static_cast<unsigned long long>(legal));
+  if (retained) atomicAdd(stats + 1, static_cast<unsigned long long>(retained));
+  if (v_loaded) atomicAdd(stats + 2, static_cast<unsigned long long>(v_loaded));
+}
+#endif
+
 struct FwdParams {
   int B, H, Hkv, L, T, G, npairs;
   int n_units;
@@ -30,6 +45,7 @@ struct FwdParams {
   uint32_t* err;      // device error word
   uint32_t* sched;    // persistent scheduler counter (zeroed before launch)
   uint64_t budget_ns;
+  unsigned long long* stats;  // call statistics (kStatsOffset) or null
 };
 
 }  // namespace mala

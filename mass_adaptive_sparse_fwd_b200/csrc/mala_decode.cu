@@ -73,6 +73,7 @@ struct DecParams {
   float* part_z;           // [B, H, S] (natural log)
   uint32_t* tickets;       // [B * Hkv]
   uint8_t* tile_mask;      // [B, H, T] or null
+  unsigned long long* stats;  // call statistics (kStatsOffset) or null
   uint32_t* err;
   uint64_t budget_ns;
 };
@@ -231,6 +232,7 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, 1)
         for (uint32_t cc = (c > NV ? c - NV : 0); cc < c; ++cc)
           mbar_wait(&sh.v_full[cc % NV], (cc / NV) & 1, drain, 5);
       }
+      stats_add(p.stats, 0, 0, c);
     }
   } else {
     // ------------------------------------------------------------------ consumers
@@ -238,6 +240,7 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, 1)
     const float NEG_INF = -INFINITY;
     const uint32_t sKa = smem_u32(sK), sVa = smem_u32(sV);
     uint32_t kc = 0, vc = 0, n_glob = 0;
+    uint32_t st_legal = 0, st_ret = 0;  // call statistics (thread 0)
     bool ok = true;
     // zero the padded heads of P once (rows >= G are never written again)
     for (int i = tid; i < kPR * 8 * (kTile + 8); i += NT) {
@@ -392,6 +395,8 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, 1)
             p.tile_mask[(static_cast<size_t>(b) * p.H + g * G + dh) * p.T + t] = k ? 1 : 0;
           // hand the decision to the V producer (ring slot must be free)
           if (tid == 0) {
+            st_legal += static_cast<uint32_t>(G);
+            st_ret += __popc(keep);
             bool free_slot = true;
             if (n_glob + n >= kPR)
               free_slot = mbar_wait(&sh.dec_empty[slot], (((n_glob + n) / kPR) - 1) & 1, ast, 11);
@@ -499,6 +504,7 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, 1)
         }
       }
     }
+    if (tid == 0) stats_add(p.stats, st_legal, st_ret, 0);
   }
   __syncthreads();
 }
@@ -544,6 +550,9 @@ mala_status decode_dispatch(const void* q, const void* K, const void* V, void* O
                             float tau, int num_splits, unsigned flags, uint8_t* ws,
                             uint8_t* tile_mask, uint64_t budget_ns, cudaStream_t stream) {
   const bool screen = (tau > 0.f) || (flags & MALA_FLAG_ALWAYS_TEST);
+  if (cudaMemsetAsync(ws + kStatsOffset, 0, 3 * sizeof(unsigned long long), stream) !=
+      cudaSuccess)
+    return MALA_ERR_CUDA;
   if (dtype == MALA_FP32)
     return fp32_decode(static_cast<const float*>(q), static_cast<const float*>(K),
                        static_cast<const float*>(V), static_cast<float*>(O), LSE, B, H, Hkv, Nk,
@@ -567,6 +576,7 @@ mala_status decode_dispatch(const void* q, const void* K, const void* V, void* O
   p.part_z = p.part_o + static_cast<size_t>(B) * H * num_splits * d;
   p.tickets = reinterpret_cast<uint32_t*>(part + ((part_bytes + 255) / 256) * 256);
   p.tile_mask = tile_mask;
+  p.stats = reinterpret_cast<unsigned long long*>(ws + kStatsOffset);
   p.err = reinterpret_cast<uint32_t*>(ws) + kHdrError;
   p.budget_ns = budget_ns;
   if (cudaMemsetAsync(p.tickets, 0, static_cast<size_t>(B) * Hkv * sizeof(uint32_t), stream) !=

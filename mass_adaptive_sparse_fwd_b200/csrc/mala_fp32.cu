@@ -39,7 +39,7 @@ __global__ void __launch_bounds__(kF32Threads)
     fp32_fwd_kernel(const float* __restrict__ Q, const float* __restrict__ K,
                     const float* __restrict__ V, float* __restrict__ O, float* __restrict__ LSE,
                     int B, int H, int Hkv, int L, int d, float scale, float tau, bool screen,
-                    uint8_t* tile_mask) {
+                    uint8_t* tile_mask, unsigned long long* stats) {
   extern __shared__ float fsm[];
   float* sK = fsm;             // [128][d]
   float* sV = fsm + kTile * d;  // [128][d]
@@ -78,8 +78,10 @@ __global__ void __launch_bounds__(kF32Threads)
     bool mine = has;
     if (screen && has && l > 0.f) mine = (rmax - m - logf(l) - theta) >= 0.f;
     const bool keep = __syncthreads_or(mine) != 0;
-    if (tile_mask && r == 0)
-      tile_mask[((static_cast<size_t>(b) * H + h) * T + i) * T + j] = keep ? 1 : 0;
+    if (r == 0) {
+      stats_add(stats, 1, keep ? 1 : 0, 0);
+      if (tile_mask) tile_mask[((static_cast<size_t>(b) * H + h) * T + i) * T + j] = keep ? 1 : 0;
+    }
     if (!keep || !has) continue;
     const float mn = fmaxf(m, rmax);
     const float alpha = expf(m - mn);
@@ -118,7 +120,8 @@ __global__ void __launch_bounds__(kF32Threads)
                        const float* __restrict__ V, const float* __restrict__ LSE,
                        const float* __restrict__ dO, const float* __restrict__ Dsum,
                        float* __restrict__ dK, float* __restrict__ dV, int B, int H, int Hkv,
-                       int L, int d, float scale, float tau, bool screen, uint8_t* tile_mask) {
+                       int L, int d, float scale, float tau, bool screen, uint8_t* tile_mask,
+                       unsigned long long* stats) {
   extern __shared__ float fsm[];
   float* sQ = fsm;               // [128][d]
   float* sdO = fsm + kTile * d;  // [128][d]
@@ -165,8 +168,10 @@ __global__ void __launch_bounds__(kF32Threads)
         if (!screen || s - sL[qq] - sT[qq] >= 0.f) mine = true;
       }
       const bool keep = __syncthreads_or(mine) != 0;
-      if (tile_mask && r == 0)
-        tile_mask[((static_cast<size_t>(b) * H + h) * T + i) * T + j] = keep ? 1 : 0;
+      if (r == 0) {
+        stats_add(stats, 1, keep ? 1 : 0, 0);
+        if (tile_mask) tile_mask[((static_cast<size_t>(b) * H + h) * T + i) * T + j] = keep ? 1 : 0;
+      }
       if (!keep || !kvalid) continue;
       for (int qq = 0; qq < kTile; ++qq) {
         const int q = i * kTile + qq;
@@ -256,7 +261,8 @@ __global__ void __launch_bounds__(kF32Threads)
     fp32_decode_split_kernel(const float* __restrict__ q, const float* __restrict__ K,
                              const float* __restrict__ V, float* __restrict__ part_o,
                              float* __restrict__ part_z, int B, int H, int Hkv, int Nk, int d,
-                             int S, float scale, float tau, bool screen, uint8_t* tile_mask) {
+                             int S, float scale, float tau, bool screen, uint8_t* tile_mask,
+                             unsigned long long* stats) {
   __shared__ float sq[128], sp[kTile], red[kTile];
   const int T = (Nk + kTile - 1) / kTile;
   const int s = blockIdx.x % S;
@@ -285,7 +291,11 @@ __global__ void __launch_bounds__(kF32Threads)
     __syncthreads();
     bool keep = true;
     if (screen && l > 0.f) keep = (rmax - m - logf(l) - theta) >= 0.f;
-    if (tile_mask && r == 0) tile_mask[(static_cast<size_t>(b) * H + h) * T + t] = keep ? 1 : 0;
+    if (r == 0) {
+      // this path loads V per head: one V tile per retained (head, tile)
+      stats_add(stats, 1, keep ? 1 : 0, keep ? 1 : 0);
+      if (tile_mask) tile_mask[(static_cast<size_t>(b) * H + h) * T + t] = keep ? 1 : 0;
+    }
     if (!keep) continue;  // uniform: every thread computed the same values
     const float mn = fmaxf(m, rmax);
     const float alpha = expf(m - mn);
@@ -341,13 +351,15 @@ cudaError_t set_smem(const void* fn, int bytes) {
 
 mala_status fp32_fwd(const float* Q, const float* K, const float* V, float* O, float* LSE, int B,
                      int H, int Hkv, int L, int d, float scale, float tau, bool screen,
-                     uint8_t* tile_mask, cudaStream_t stream) {
+                     uint8_t* ws, uint8_t* tile_mask, cudaStream_t stream) {
   const int T = (L + kTile - 1) / kTile;
   const int smem = 2 * kTile * d * static_cast<int>(sizeof(float));
+  unsigned long long* stats =
+      ws ? reinterpret_cast<unsigned long long*>(ws + kStatsOffset) : nullptr;
   if (set_smem(reinterpret_cast<const void*>(fp32_fwd_kernel), smem) != cudaSuccess)
     return MALA_ERR_CUDA;
   fp32_fwd_kernel<<<B * H * T, kF32Threads, smem, stream>>>(Q, K, V, O, LSE, B, H, Hkv, L, d,
-                                                            scale, tau, screen, tile_mask);
+                                                            scale, tau, screen, tile_mask, stats);
   return cudaGetLastError() == cudaSuccess ? MALA_OK : MALA_ERR_CUDA;
 }
 
@@ -366,7 +378,8 @@ mala_status fp32_bwd(const float* Q, const float* K, const float* V, const float
       set_smem(reinterpret_cast<const void*>(fp32_bwd_q_kernel), smem_q) != cudaSuccess)
     return MALA_ERR_CUDA;
   fp32_bwd_kv_kernel<<<B * Hkv * T, kF32Threads, smem_kv, stream>>>(
-      Q, K, V, LSE, dO, Dsum, dK, dV, B, H, Hkv, L, d, scale, tau, screen, tile_mask);
+      Q, K, V, LSE, dO, Dsum, dK, dV, B, H, Hkv, L, d, scale, tau, screen, tile_mask,
+      reinterpret_cast<unsigned long long*>(ws + kStatsOffset));
   fp32_bwd_q_kernel<<<B * H * T, kF32Threads, smem_q, stream>>>(Q, K, V, LSE, dO, Dsum, dQ, B, H,
                                                                 Hkv, L, d, scale, tau, screen);
   return cudaGetLastError() == cudaSuccess ? MALA_OK : MALA_ERR_CUDA;
@@ -378,7 +391,8 @@ mala_status fp32_decode(const float* q, const float* K, const float* V, float* O
   float* part_o = reinterpret_cast<float*>(ws + kWorkspaceHeader);
   float* part_z = part_o + static_cast<size_t>(B) * H * S * d;
   fp32_decode_split_kernel<<<B * H * S, kF32Threads, 0, stream>>>(
-      q, K, V, part_o, part_z, B, H, Hkv, Nk, d, S, scale, tau, screen, tile_mask);
+      q, K, V, part_o, part_z, B, H, Hkv, Nk, d, S, scale, tau, screen, tile_mask,
+      reinterpret_cast<unsigned long long*>(ws + kStatsOffset));
   fp32_decode_merge_kernel<<<B * H, 128, 0, stream>>>(part_o, part_z, O, LSE, B * H, S, d);
   return cudaGetLastError() == cudaSuccess ? MALA_OK : MALA_ERR_CUDA;
 }

@@ -292,6 +292,7 @@ __global__ void __launch_bounds__(384, 1)
     const uint32_t tO = tb + 256 + s * D + lane_off;
     const float NEG_INF = -INFINITY;
     uint32_t ns = 0, npv = 0;
+    uint32_t st_legal = 0, st_ret = 0;  // call statistics (row-0 thread of the slot)
     bool ok = true;
     for (uint32_t k = 0; ok; ++k) {
       const int ring = k & 1;
@@ -355,8 +356,12 @@ __global__ void __launch_bounds__(384, 1)
           keep = named_bar_or(1 + s, 128, mine);
           if (*ast.flag) { ok = false; break; }
         }
-        if (p.tile_mask && r == 0)
-          p.tile_mask[((static_cast<size_t>(w.b) * p.H + h) * p.T + w.i) * p.T + j] = keep ? 1 : 0;
+        if (r == 0) {
+          ++st_legal;
+          st_ret += keep ? 1u : 0u;
+          if (p.tile_mask)
+            p.tile_mask[((static_cast<size_t>(w.b) * p.H + h) * p.T + w.i) * p.T + j] = keep ? 1 : 0;
+        }
         if (!keep) {
           if (r == 0) sh.dec[s] = 0;
           tc_fence_before();
@@ -449,6 +454,7 @@ __global__ void __launch_bounds__(384, 1)
       if (valid) p.LSE[(static_cast<size_t>(w.b) * p.H + h) * p.L + q] = (m2 + __log2f(l)) * kLn2;
       tc_fence_before();
     }
+    if (r == 0) stats_add(p.stats, st_legal, st_ret, 0);
   }
 
   tc_fence_before();

@@ -24,10 +24,16 @@ MALA_BF16, MALA_FP32 = 0, 1
 MALA_FLAG_ALWAYS_TEST = 1
 TILE = 128
 
-EXPORTED = ("mala_fwd", "mala_bwd", "mala_decode", "mala_decode_noalloc", "mala_fwd_workspace_bytes",
+EXPORTED = ("mala_fwd", "mala_bwd", "mala_decode", "mala_decode_noalloc", "mala_get_stats",
+            "mala_fwd_workspace_bytes",
             "mala_bwd_workspace_bytes", "mala_decode_workspace_bytes", "mala_decode_num_splits",
             "mala_read_device_error", "mala_set_wait_budget_ns", "mala_status_string",
             "mala_version")
+
+
+class MalaStats(ctypes.Structure):
+    _fields_ = [("legal_tiles", ctypes.c_uint64), ("retained_tiles", ctypes.c_uint64),
+                ("v_tiles_loaded", ctypes.c_uint64)]
 
 
 class MalaError(RuntimeError):
@@ -64,6 +70,8 @@ def load_library(path: str = _LIB_PATH) -> ctypes.CDLL:
     lib.mala_decode_num_splits.restype = ci
     lib.mala_read_device_error.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_uint32), ci]
     lib.mala_set_wait_budget_ns.argtypes = [ctypes.c_uint64]
+    lib.mala_get_stats.argtypes = [vp, vp, ctypes.POINTER(MalaStats)]
+    lib.mala_get_stats.restype = ci
     lib.mala_status_string.argtypes = [ci]
     lib.mala_status_string.restype = ctypes.c_char_p
     lib.mala_version.restype = ci
@@ -197,6 +205,16 @@ def read_device_error(workspace: torch.Tensor, clear: bool = True, stream=None) 
            _lib.mala_read_device_error(_ptr(workspace), _stream(stream), ctypes.byref(out),
                                        int(clear)))
     return out.value
+
+
+def get_stats(workspace: torch.Tensor, stream=None) -> dict:
+    """Work counters of the last call that ran on `workspace` (synchronises the stream):
+    legal tiles tested, retained tiles and, for decode, V tiles loaded."""
+    out = MalaStats()
+    _check("mala_get_stats", _lib.mala_get_stats(_ptr(workspace), _stream(stream),
+                                                 ctypes.byref(out)))
+    return {"legal_tiles": out.legal_tiles, "retained_tiles": out.retained_tiles,
+            "v_tiles_loaded": out.v_tiles_loaded}
 
 
 def set_wait_budget_ns(ns: int):

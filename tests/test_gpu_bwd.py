@@ -38,9 +38,13 @@ def run_fwd_bwd(mala, inp, w, tau, flags=0):
     torch.cuda.synchronize()
     assert mala.read_device_error(wsf) == 0
     assert mala.read_device_error(wsb) == 0
+    # the backward call's work counters agree with its tile decisions
+    legal = P.fwd_legal(B, H, T)
+    bm = bmask.cpu().numpy()
+    st = mala.get_stats(wsb)
+    assert st["legal_tiles"] == legal.sum() and st["retained_tiles"] == (bm[legal] == 1).sum()
     cpu = lambda t: t.float().cpu().numpy()
-    return (cpu(O), cpu(LSE), fmask.cpu().numpy(), cpu(dQ), cpu(dK), cpu(dV),
-            bmask.cpu().numpy())
+    return (cpu(O), cpu(LSE), fmask.cpu().numpy(), cpu(dQ), cpu(dK), cpu(dV), bm)
 
 
 def check_bwd(orc, mala, w, inp, tau, kv_units=None, q_units=None, flags=0):

@@ -43,6 +43,13 @@ def check_decode(orc, mala, inp, scale, tau, S, dtype="bf16", units=None, flags=
     assert mala.read_device_error(ws) == 0
     O, LSE, mask = O.float().cpu().numpy(), LSE.cpu().numpy(), mask.cpu().numpy()
     assert np.isin(mask, (0, 1)).all()
+    # the call's work counters: tested and retained (b, h, tile) pairs, V tiles fetched
+    # (per KV group on the tensor-core path, per head on the fp32 path)
+    st = mala.get_stats(ws)
+    assert st["legal_tiles"] == mask.size and st["retained_tiles"] == mask.sum()
+    v_tiles = mask.sum() if dtype == "fp32" else \
+        mask.reshape(B, Hkv, H // Hkv, T).max(axis=2).sum()
+    assert st["v_tiles_loaded"] == v_tiles
     oO, oLSE, _, omargin, _, _ = orc.mala_decode(inp["q"], inp["K"], inp["V"], scale, tau, S,
                                                   units=units, force=mask.astype(np.int8))
     sel = np.isfinite(oLSE)

@@ -28,7 +28,12 @@ def run_fwd(mala, inp, w, tau, flags=0):
     O, LSE = mala.mala_fwd(Q, K, V, w.scale, tau, flags=flags, workspace=ws, tile_mask=mask)
     torch.cuda.synchronize()
     assert mala.read_device_error(ws) == 0
-    return O.float().cpu().numpy(), LSE.cpu().numpy(), mask.cpu().numpy()
+    mask = mask.cpu().numpy()
+    # the call's work counters agree with its tile decisions
+    legal = P.fwd_legal(B, H, T)
+    st = mala.get_stats(ws)
+    assert st["legal_tiles"] == legal.sum() and st["retained_tiles"] == (mask[legal] == 1).sum()
+    return O.float().cpu().numpy(), LSE.cpu().numpy(), mask
 
 
 def check_fwd(orc, mala, w, inp, tau, units=None, flags=0):

@@ -85,6 +85,8 @@ def test_invalid_arguments_are_rejected_before_any_launch(lib):
     # backward: bad dtype code
     assert L.mala_bwd(vp(), vp(), vp(), vp(), vp(), vp(), vp(), vp(), vp(), 1, 4, 2, 128, 128, 7,
                       0.1, 1.0, 0, None, 0, None, None) == 1
+    # statistics need a workspace and an output
+    assert L.mala_get_stats(None, None, None) == 1
     # workspace too small (checked before any CUDA call)
     assert L.mala_fwd(vp(), vp(), vp(), vp(), vp(), 1, 4, 2, 128, 128, 0, 0.1, 1.0, 0, vp(), 8,
                       None, None) == 5
