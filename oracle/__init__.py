@@ -56,8 +56,10 @@ def _load():
                                          vp, ci, vp, ci, vp, vp, vp, vp, vp, vp]
             lib.orc_mala_decode.argtypes = [vp, vp, vp, ci, ci, ci, ci, ci, cd, cd, ci, ci, vp,
                                             ci, vp, vp, vp, vp, vp, vp, vp]
+            lib.orc_mala_prefill.argtypes = [vp, vp, vp, ci, ci, ci, ci, ci, ci, cd, cd, ci, vp,
+                                             ci, vp, vp, vp, vp, vp]
             for name in ("orc_dense_fwd", "orc_dense_bwd", "orc_mala_fwd", "orc_mala_fwd_setsum",
-                         "orc_mala_bwd", "orc_mala_decode"):
+                         "orc_mala_bwd", "orc_mala_decode", "orc_mala_prefill"):
                 getattr(lib, name).restype = ctypes.c_int
             _lib = lib
     return _lib
@@ -135,6 +137,29 @@ def mala_fwd(Q, K, V, scale, tau, blk=128, units=None, force=None):
     rc = _load().orc_mala_fwd(_p(Q), _p(K), _p(V), B, H, Hkv, L, d, float(scale), float(tau), blk,
                               _p(u), n, _p(force), _p(O), _p(LSE), _p(mask), _p(margin))
     _check(rc, "mala_fwd")
+    return O, LSE, mask, margin
+
+
+def mala_prefill(Q, K, V, scale, tau, blk=128, units=None, force=None):
+    """Chunked-prefill forward: Q [B,Nq,H,d] are the last Nq positions of a sequence whose
+    keys K, V [B,Nk,Hkv,d] (Nk >= Nq) include them; row q sits at position Nk - Nq + q.
+    Returns (O, LSE, mask, margin) with mask / margin [B,H,Tq,Tk]."""
+    Q, K, V = _f32(Q), _f32(K), _f32(V)
+    B, Nq, H, d = Q.shape
+    Nk, Hkv = K.shape[1], K.shape[2]
+    Tq, Tk = n_tiles(Nq, blk), n_tiles(Nk, blk)
+    O = np.full(Q.shape, np.nan)
+    LSE = np.full((B, H, Nq), np.nan)
+    mask = np.full((B, H, Tq, Tk), -1, dtype=np.int8)
+    margin = np.full((B, H, Tq, Tk), np.nan)
+    u, n = _units(units, 3)
+    if force is not None:
+        force = np.ascontiguousarray(force, dtype=np.int8)
+        assert force.shape == (B, H, Tq, Tk)
+    rc = _load().orc_mala_prefill(_p(Q), _p(K), _p(V), B, H, Hkv, Nq, Nk, d, float(scale),
+                                  float(tau), blk, _p(u), n, _p(force), _p(O), _p(LSE), _p(mask),
+                                  _p(margin))
+    _check(rc, "mala_prefill")
     return O, LSE, mask, margin
 
 

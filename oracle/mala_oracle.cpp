@@ -10,6 +10,8 @@
 //   §2.4  split-KV decoding with per-split partial normalisers
 //   App. A, Algorithm 1 (forward) and Algorithm 2 (backward); A.1 traversal order
 //   App. B, Proposition 1 (the invariants the tests check)
+//   §2.3  the same forward serves inference prefill: orc_mala_prefill takes a chunk of
+//         queries at the end of a longer key sequence (causal offset Nk - Nq)
 //
 // Conventions (each one a reading of the page, listed in the design doc):
 //   * scores s = scale * <q, k>, natural exp / log (§2.1 absorbs the scale into Q)
@@ -374,6 +376,92 @@ void bwd_q_block(const BwdCtx& C, int b, int h, int i, const signed char* force,
   }
 }
 
+// ---------------------------------------------------------------------------
+// Chunked prefill: the forward of Algorithm 1 for a chunk of Nq queries that are the
+// last Nq positions of a sequence of Nk >= Nq keys ("the same forward operator serves
+// ... inference prefill", §2.3).  Query row q (0-based in the chunk) sits at absolute
+// position p = off + q, off = Nk - Nq; it attends to keys k <= p, and L_q = p + 1.
+// Query block i holds chunk rows [i*blk, (i+1)*blk); it visits the key blocks that hold
+// a legal key of one of its rows, from the last one (the block of its last row's
+// position) down to 0.
+struct PDims {
+  int B, H, Hkv, Nq, Nk, off, d, G, Tq, Tk;
+  long long q_off(int b, int q, int h) const { return (((long long)b * Nq + q) * H + h) * d; }
+  long long kv_off(int b, int k, int g) const { return (((long long)b * Nk + k) * Hkv + g) * d; }
+  long long lse_off(int b, int h, int q) const { return ((long long)b * H + h) * Nq + q; }
+  long long tile_off(int b, int h, int i, int j) const {
+    return (((long long)b * H + h) * Tq + i) * Tk + j;
+  }
+};
+
+void prefill_block(const PDims& D, const float* Q, const float* K, const float* V, double scale,
+                   double tau, int blk, int b, int h, int i, const signed char* force, double* O,
+                   double* LSE, signed char* mask, double* margin) {
+  const int g = h / D.G;
+  const int q0 = i * blk;
+  const int q1 = std::min(D.Nq, q0 + blk);
+  const int nq = q1 - q0;
+  std::vector<double> m(nq, -kInf), l(nq, 0.0), acc((size_t)nq * D.d, 0.0), theta(nq);
+  for (int r = 0; r < nq; ++r) theta[r] = log_threshold(tau, (double)(D.off + q0 + r + 1));
+  std::vector<double> S((size_t)nq * blk), rowmax(nq);
+  std::vector<char> has_key(nq);
+  const int j_last = (D.off + q1 - 1) / blk;
+  for (int j = j_last; j >= 0; --j) {
+    const int k0 = j * blk;
+    const int k1 = std::min(D.Nk, k0 + blk);
+    for (int r = 0; r < nq; ++r) {
+      const int pos = D.off + q0 + r;
+      rowmax[r] = -kInf;
+      has_key[r] = 0;
+      const float* qv = Q + D.q_off(b, q0 + r, h);
+      for (int k = k0; k < k1; ++k) {
+        double sc = -kInf;
+        if (k <= pos) {
+          sc = scale * dot(qv, K + D.kv_off(b, k, g), D.d);
+          has_key[r] = 1;
+          if (sc > rowmax[r]) rowmax[r] = sc;
+        }
+        S[(size_t)r * blk + (k - k0)] = sc;
+      }
+    }
+    double X = -kInf;  // Eq. (3) over the rows with a legal key in this tile
+    for (int r = 0; r < nq; ++r) {
+      if (!has_key[r]) continue;
+      const double x = (l[r] == 0.0) ? kInf : rowmax[r] - m[r] - std::log(l[r]) - theta[r];
+      if (x > X) X = x;
+    }
+    bool retain = (X >= 0.0);
+    const long long to = D.tile_off(b, h, i, j);
+    if (force && force[to] >= 0) retain = (force[to] != 0);
+    if (mask) mask[to] = retain ? 1 : 0;
+    if (margin) margin[to] = X;
+    if (!retain) continue;
+    for (int r = 0; r < nq; ++r) {
+      if (!has_key[r]) continue;
+      const double mn = std::max(m[r], rowmax[r]);
+      const double alpha = std::exp(m[r] - mn);
+      double psum = 0.0;
+      double* a = &acc[(size_t)r * D.d];
+      for (int c = 0; c < D.d; ++c) a[c] *= alpha;
+      for (int k = k0; k < k1; ++k) {
+        const double sc = S[(size_t)r * blk + (k - k0)];
+        if (sc == -kInf) continue;
+        const double pr = std::exp(sc - mn);
+        psum += pr;
+        const float* vv = V + D.kv_off(b, k, g);
+        for (int c = 0; c < D.d; ++c) a[c] += pr * (double)vv[c];
+      }
+      l[r] = alpha * l[r] + psum;
+      m[r] = mn;
+    }
+  }
+  for (int r = 0; r < nq; ++r) {
+    double* o = O + D.q_off(b, q0 + r, h);
+    for (int c = 0; c < D.d; ++c) o[c] = acc[(size_t)r * D.d + c] / l[r];
+    LSE[D.lse_off(b, h, q0 + r)] = m[r] + std::log(l[r]);
+  }
+}
+
 }  // namespace
 
 extern "C" {
@@ -460,6 +548,30 @@ int orc_mala_fwd(const float* Q, const float* K, const float* V, int B, int H, i
       b = (int)(u / ((long long)H * D.T)); h = (int)((u / D.T) % H); i = (int)(u % D.T);
     }
     mala_fwd_block(D, Q, K, V, scale, tau, blk, b, h, i, force, O, LSE, mask, margin);
+  }
+  return 0;
+}
+
+// Chunked prefill forward (see prefill_block).  Q, O [B, Nq, H, d]; K, V [B, Nk, Hkv, d];
+// LSE [B, H, Nq]; mask / margin [B, H, Tq, Tk].  units: (b, h, i) or NULL for all.
+int orc_mala_prefill(const float* Q, const float* K, const float* V, int B, int H, int Hkv,
+                     int Nq, int Nk, int d, double scale, double tau, int blk, const int* units,
+                     int n_units, const signed char* force, double* O, double* LSE,
+                     signed char* mask, double* margin) {
+  if (bad_dims(B, H, Hkv, Nq, d, blk) || Nk < Nq || !(tau >= 0.0)) return -1;
+  PDims D;
+  D.B = B; D.H = H; D.Hkv = Hkv; D.Nq = Nq; D.Nk = Nk; D.off = Nk - Nq; D.d = d;
+  D.G = H / Hkv; D.Tq = (Nq + blk - 1) / blk; D.Tk = (Nk + blk - 1) / blk;
+  const long long n = units ? n_units : (long long)B * H * D.Tq;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (long long u = 0; u < n; ++u) {
+    int b, h, i;
+    if (units) {
+      b = units[3 * u]; h = units[3 * u + 1]; i = units[3 * u + 2];
+    } else {
+      b = (int)(u / ((long long)H * D.Tq)); h = (int)((u / D.Tq) % H); i = (int)(u % D.Tq);
+    }
+    prefill_block(D, Q, K, V, scale, tau, blk, b, h, i, force, O, LSE, mask, margin);
   }
   return 0;
 }

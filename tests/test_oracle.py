@@ -545,3 +545,142 @@ def test_synth_round_bf16_ties_to_even():
     r = synth.round_bf16(x)
     np.testing.assert_array_equal(r[:3], [1.0, 1.0 + 2 ** -6, -1.5])
     np.testing.assert_array_equal(r, torch.from_numpy(x).to(torch.bfloat16).float().numpy())
+
+
+# ---------------------------------------------------------------------------- chunked prefill
+# A chunk of Nq queries at the end of a sequence of Nk keys (§2.3: the forward serves
+# inference prefill); row q sits at position Nk - Nq + q.
+
+
+def _allowed_offset(B, H, Nq, Nk):
+    off = Nk - Nq
+    a = np.arange(Nk)[None, :] <= (off + np.arange(Nq))[:, None]
+    return np.broadcast_to(a, (B, H, Nq, Nk)).copy()
+
+
+def _sdpa_offset(Q, K, V, scale, allowed):
+    """Softmax attention over an explicit key mask [B,H,Nq,Nk] via torch in fp64."""
+    G = Q.shape[2] // K.shape[2]
+    q, k, v = _torch_bhld(Q), _expand_kv(_torch_bhld(K), G), _expand_kv(_torch_bhld(V), G)
+    m = torch.from_numpy(allowed)
+    out = F.scaled_dot_product_attention(q, k, v, attn_mask=m, scale=scale)
+    s = (q @ k.transpose(-1, -2)) * scale
+    lse = torch.logsumexp(s.masked_fill(~m, float("-inf")), dim=-1)
+    return out.permute(0, 2, 1, 3).numpy(), lse.numpy()
+
+
+def _rand_chunk(B, Nq, Nk, H, Hkv, d, seed, peak=0.0):
+    Q, K, V, _ = _rand(B, Nk, H, Hkv, d, seed, peak=peak)
+    return np.ascontiguousarray(Q[:, Nk - Nq:]), K, V, Q
+
+
+def test_prefill_full_length_equals_forward(orc):
+    Q, K, V, _ = _rand(2, 70, 4, 2, 16, seed=41, peak=4.0)
+    a = orc.mala_prefill(Q, K, V, 0.25, 1.0, blk=16)
+    b = orc.mala_fwd(Q, K, V, 0.25, 1.0, blk=16)
+    for x, y in zip(a, b):
+        np.testing.assert_array_equal(x, y)
+
+
+def test_prefill_aligned_offset_equals_tail_of_forward(orc):
+    # off = 48 = 3 blocks of 16: the chunk's query blocks are the forward's blocks 3..5
+    Qc, K, V, Qf = _rand_chunk(1, 48, 96, 2, 1, 16, seed=42, peak=5.0)
+    O, LSE, mask, margin = orc.mala_prefill(Qc, K, V, 0.25, 1.0, blk=16)
+    Of, LSEf, maskf, marginf = orc.mala_fwd(Qf, K, V, 0.25, 1.0, blk=16)
+    np.testing.assert_array_equal(O, Of[:, 48:])
+    np.testing.assert_array_equal(LSE, LSEf[:, :, 48:])
+    np.testing.assert_array_equal(mask, maskf[:, :, 3:])
+    np.testing.assert_array_equal(margin, marginf[:, :, 3:])
+    assert (mask == 0).any()
+
+
+@pytest.mark.parametrize("Nq,Nk", [(37, 101), (16, 16), (1, 50), (64, 77)])
+def test_prefill_tau0_is_dense_with_offset(orc, Nq, Nk):
+    Qc, K, V, _ = _rand_chunk(2, Nq, Nk, 4, 2, 16, seed=43 + Nq)
+    O, LSE, mask, _ = orc.mala_prefill(Qc, K, V, 0.3, 0.0, blk=16)
+    O_t, LSE_t = _sdpa_offset(Qc, K, V, 0.3, _allowed_offset(2, 4, Nq, Nk))
+    np.testing.assert_allclose(O, O_t, atol=1e-12)
+    np.testing.assert_allclose(LSE, LSE_t, atol=1e-12)
+    assert (mask[mask >= 0] == 1).all()
+
+
+def _check_eq3_offset(Q, K, scale, tau, blk, mask):
+    """Brute force of Eq. (3) with the causal offset: every decision re-derived from raw
+    scores and the recorded decisions of the tiles visited before it."""
+    B, Nq, H, _ = Q.shape
+    Nk = K.shape[1]
+    off = Nk - Nq
+    G = H // K.shape[2]
+    s = np.einsum("bqhd,bkhd->bhqk", Q.astype(np.float64),
+                  np.repeat(K.astype(np.float64), G, axis=2)) * scale
+    s[~_allowed_offset(B, H, Nq, Nk)] = -np.inf
+    Tq = mask.shape[2]
+    n = 0
+    for b in range(B):
+        for h in range(H):
+            for i in range(Tq):
+                rows = np.arange(i * blk, min(Nq, (i + 1) * blk))
+                pos = off + rows
+                Z = np.zeros(len(rows))
+                for j in range(pos[-1] // blk, -1, -1):
+                    cols = np.arange(j * blk, min(Nk, (j + 1) * blk))
+                    st = s[b, h][np.ix_(rows, cols)]
+                    legal = np.isfinite(st)
+                    top = np.where(legal, st, -np.inf).max(axis=1)
+                    has = legal.any(axis=1)
+                    with np.errstate(divide="ignore", over="ignore"):
+                        ratio = np.where(Z > 0, np.exp(top) / np.where(Z > 0, Z, 1), np.inf)
+                    retain = bool((has & (ratio >= tau / (pos + 1))).any())
+                    assert retain == (mask[b, h, i, j] == 1), (b, h, i, j)
+                    n += 1
+                    if retain:
+                        Z += np.where(legal, np.exp(np.where(legal, st, 0.0)), 0.0).sum(axis=1)
+                assert (mask[b, h, i, pos[-1] // blk + 1:] == -1).all()  # not legal
+    return n
+
+
+@pytest.mark.parametrize("tau", [0.5, 1.0, 4.0])
+def test_prefill_decisions_brute_force(orc, tau):
+    Qc, K, V, _ = _rand_chunk(1, 45, 117, 2, 1, 16, seed=44, peak=6.0)
+    _, _, mask, _ = orc.mala_prefill(Qc, K, V, 0.25, tau, blk=8)
+    assert _check_eq3_offset(Qc, K, 0.25, tau, 8, mask) > 0
+    assert (mask == 0).any()
+
+
+def test_prefill_output_is_softmax_over_retained_tiles(orc):
+    Qc, K, V, _ = _rand_chunk(2, 40, 93, 4, 2, 16, seed=45, peak=3.0)
+    O, LSE, mask, _ = orc.mala_prefill(Qc, K, V, 0.25, 1.0, blk=16)
+    keep = np.kron(np.where(mask == 1, 1, 0), np.ones((16, 16), int))[:, :, :40, :93] > 0
+    allowed = _allowed_offset(2, 4, 40, 93) & keep
+    O_t, LSE_t = _sdpa_offset(Qc, K, V, 0.25, allowed)
+    np.testing.assert_allclose(O, O_t, atol=1e-12)
+    np.testing.assert_allclose(LSE, LSE_t, atol=1e-12)
+
+
+def test_prefill_huge_tau_keeps_the_blocks_own_key_tiles(orc):
+    # off = 53 is not a multiple of 16: a query block spans two key tiles, and each of
+    # them is some row's first legal tile (l = 0), so both are retained; older tiles go
+    Nq, Nk, blk = 40, 93, 16
+    Qc, K, V, _ = _rand_chunk(1, Nq, Nk, 2, 2, 8, seed=46)
+    O, LSE, mask, _ = orc.mala_prefill(Qc, K, V, 0.3, 1e30, blk=blk)
+    off = Nk - Nq
+    first_tile = ((off + (np.arange(Nq) // blk) * blk) // blk)  # tile of the block's first row
+    allowed = _allowed_offset(1, 2, Nq, Nk) & (np.arange(Nk)[None, :] >= first_tile[:, None] * blk)
+    O_t, LSE_t = _sdpa_offset(Qc, K, V, 0.3, allowed)
+    np.testing.assert_allclose(O, O_t, atol=1e-12)
+    np.testing.assert_allclose(LSE, LSE_t, atol=1e-12)
+    for i in range(mask.shape[2]):
+        jf = (off + i * blk) // blk
+        jl = (off + min(Nq, (i + 1) * blk) - 1) // blk
+        assert (mask[:, :, i, jf:jl + 1] == 1).all() and (mask[:, :, i, :jf] == 0).all()
+
+
+def test_prefill_units_match_full(orc):
+    Qc, K, V, _ = _rand_chunk(2, 50, 130, 4, 2, 16, seed=47, peak=4.0)
+    full = orc.mala_prefill(Qc, K, V, 0.25, 1.0, blk=16)
+    units = [(1, 3, 3), (0, 0, 0), (1, 2, 1)]
+    part = orc.mala_prefill(Qc, K, V, 0.25, 1.0, blk=16, units=units)
+    for b, h, i in units:
+        rows = slice(i * 16, min(50, (i + 1) * 16))
+        np.testing.assert_array_equal(part[0][b, rows, h], full[0][b, rows, h])
+        np.testing.assert_array_equal(part[2][b, h, i], full[2][b, h, i])
