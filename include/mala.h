@@ -77,6 +77,25 @@ mala_status mala_fwd(const void* Q, const void* K, const void* V, void* O, float
                      uint8_t* tile_mask, void* stream);
 
 /*
+ * mala_fwd_prefill - MALA forward of a prefill chunk (chunked prefill).
+ * "MassAlloc Attention", §2.3 (the same forward serves inference prefill) with the
+ * forward rules of §2.2 / Algorithm 1.  The N_q queries are the last N_q positions of a
+ * sequence of N_k >= N_q keys that already holds them (the KV cache including the chunk):
+ * query row q sits at position p = N_k - N_q + q, attends to keys k <= p, and is tested
+ * with L_q = p + 1.  Query block i (rows [128 i, 128 i + 128)) visits the key blocks that
+ * hold a legal key of one of its rows, from the last one down to 0; when N_k - N_q is not
+ * a multiple of 128 the block straddles two key blocks, and both are masked per row.
+ *   Q [B,N_q,H,d], K/V [B,N_k,H_kv,d] in; O [B,N_q,H,d], LSE [B,H,N_q] float32 out.
+ *   tile_mask (optional) is [B, H, ceil(N_q/128), ceil(N_k/128)], entry [b][h][i][j].
+ *   N_q == N_k is exactly mala_fwd.  Workspace: mala_fwd_workspace_bytes(B,H,H_kv,N_q,d,.).
+ *   Errors as mala_fwd; N_q > N_k is MALA_ERR_INVALID_ARG.
+ */
+mala_status mala_fwd_prefill(const void* Q, const void* K, const void* V, void* O, float* LSE,
+                             int B, int H, int H_kv, int N_q, int N_k, int d, int dtype,
+                             float scale, float tau, unsigned flags, void* workspace,
+                             size_t workspace_bytes, uint8_t* tile_mask, void* stream);
+
+/*
  * mala_bwd - MALA backward.
  * "MassAlloc Attention", §2.2 (offline sparse probability, Eq. (4)), App. A
  * Algorithm 2 and A.1 (fused backward execution).  O and LSE are the forward's

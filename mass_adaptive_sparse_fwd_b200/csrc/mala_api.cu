@@ -28,7 +28,7 @@ mala_status decode_dispatch(const void* q, const void* K, const void* V, void* O
 size_t decode_workspace_bytes(int B, int H, int Hkv, int Nk, int d, int dtype, int num_splits);
 int decode_auto_splits(int B, int Hkv, int Nk);
 mala_status fp32_fwd(const float* Q, const float* K, const float* V, float* O, float* LSE, int B,
-                     int H, int Hkv, int L, int d, float scale, float tau, bool screen,
+                     int H, int Hkv, int L, int Lk, int d, float scale, float tau, bool screen,
                      uint8_t* ws, uint8_t* tile_mask, cudaStream_t stream);
 
 // ---------------------------------------------------------------------------- shared host helpers
@@ -168,17 +168,26 @@ size_t mala_fwd_workspace_bytes(int B, int H, int H_kv, int L, int d, int dtype)
   return kWorkspaceHeader;
 }
 
-mala_status mala_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE, int B,
-                     int H, int H_kv, int L, int d, int dtype, float scale, float tau,
-                     unsigned flags, void* workspace, size_t workspace_bytes,
-                     uint8_t* tile_mask, void* stream) {
+}  // extern "C"
+
+namespace mala {
+namespace {
+
+// The forward for L query rows that are the last L of Lk key positions (Lk == L: the
+// ordinary causal forward; Lk > L: a prefill chunk with causal offset Lk - L).
+mala_status run_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE, int B,
+                    int H, int H_kv, int L, int Lk, int d, int dtype, float scale, float tau,
+                    unsigned flags, void* workspace, size_t workspace_bytes, uint8_t* tile_mask,
+                    void* stream) {
   if (!common_args_ok(B, H, H_kv, L, d, dtype, scale, tau)) return MALA_ERR_INVALID_ARG;
+  if (Lk < L) return MALA_ERR_INVALID_ARG;
   if (!Q || !K || !V || !O || !LSE) return MALA_ERR_INVALID_ARG;
   if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O))
     return MALA_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const bool screen = (tau > 0.f) || (flags & MALA_FLAG_ALWAYS_TEST);
   const int T = (L + kTile - 1) / kTile;
+  const int Tk = (Lk + kTile - 1) / kTile;
   if (dtype == MALA_FP32) {
     if (d > 128) return MALA_ERR_UNSUPPORTED;
     // this path needs no scratch; a caller's workspace only receives the call statistics
@@ -192,17 +201,17 @@ mala_status mala_fwd(const void* Q, const void* K, const void* V, void* O, float
         return MALA_ERR_CUDA;
     }
     return fp32_fwd(static_cast<const float*>(Q), static_cast<const float*>(K),
-                    static_cast<const float*>(V), static_cast<float*>(O), LSE, B, H, H_kv, L, d,
-                    scale, tau, screen, ws, tile_mask, st);
+                    static_cast<const float*>(V), static_cast<float*>(O), LSE, B, H, H_kv, L, Lk,
+                    d, scale, tau, screen, ws, tile_mask, st);
   }
   if (d != 64 && d != 128) return MALA_ERR_UNSUPPORTED;
-  if ((long long)B * L > (1ll << 31) || (long long)B * H * T > (1ll << 30))
+  if ((long long)B * Lk > (1ll << 31) || (long long)B * H * T > (1ll << 30))
     return MALA_ERR_UNSUPPORTED;
   if (workspace && workspace_bytes < mala_fwd_workspace_bytes(B, H, H_kv, L, d, dtype))
     return MALA_ERR_WORKSPACE;
   CUtensorMap tq, tk, tv;
-  if (!make_tile_map(&tq, Q, d, H, L, B) || !make_tile_map(&tk, K, d, H_kv, L, B) ||
-      !make_tile_map(&tv, V, d, H_kv, L, B))
+  if (!make_tile_map(&tq, Q, d, H, L, B) || !make_tile_map(&tk, K, d, H_kv, Lk, B) ||
+      !make_tile_map(&tv, V, d, H_kv, Lk, B))
     return MALA_ERR_CUDA;
   const size_t need = mala_fwd_workspace_bytes(B, H, H_kv, L, d, dtype);
   return with_workspace(workspace, workspace_bytes, need, st, [&](uint8_t* ws) -> mala_status {
@@ -212,6 +221,7 @@ mala_status mala_fwd(const void* Q, const void* K, const void* V, void* O, float
       return MALA_ERR_CUDA;
     FwdParams p;
     p.B = B; p.H = H; p.Hkv = H_kv; p.L = L; p.T = T; p.G = H / H_kv;
+    p.Lk = Lk; p.Tk = Tk; p.off = Lk - L;
     p.npairs = (p.G + 1) / 2;
     p.n_units = T * B * H_kv * p.npairs;
     p.scale_log2 = scale * kLog2e;
@@ -225,6 +235,28 @@ mala_status mala_fwd(const void* Q, const void* K, const void* V, void* O, float
     cudaError_t e = launch_fwd_bf16(tq, tk, tv, p, d, screen, grid, st);
     return e == cudaSuccess ? MALA_OK : MALA_ERR_CUDA;
   });
+}
+
+}  // namespace
+}  // namespace mala
+
+extern "C" {
+
+mala_status mala_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE, int B,
+                     int H, int H_kv, int L, int d, int dtype, float scale, float tau,
+                     unsigned flags, void* workspace, size_t workspace_bytes,
+                     uint8_t* tile_mask, void* stream) {
+  return run_fwd(Q, K, V, O, LSE, B, H, H_kv, L, L, d, dtype, scale, tau, flags, workspace,
+                 workspace_bytes, tile_mask, stream);
+}
+
+mala_status mala_fwd_prefill(const void* Q, const void* K, const void* V, void* O, float* LSE,
+                             int B, int H, int H_kv, int N_q, int N_k, int d, int dtype,
+                             float scale, float tau, unsigned flags, void* workspace,
+                             size_t workspace_bytes, uint8_t* tile_mask, void* stream) {
+  if (N_k <= 0 || N_q > N_k) return MALA_ERR_INVALID_ARG;
+  return run_fwd(Q, K, V, O, LSE, B, H, H_kv, N_q, N_k, d, dtype, scale, tau, flags, workspace,
+                 workspace_bytes, tile_mask, stream);
 }
 
 size_t mala_bwd_workspace_bytes(int B, int H, int H_kv, int L, int d, int dtype) {

@@ -362,8 +362,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const int tw = tid - 128 - 128 * wg;    // 0..127 within the warpgroup
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
     const float NEG_INF = -INFINITY;
-    uint32_t ntile = 0, nret = 0;
-    uint32_t st_legal = 0, st_ret = 0;  // call statistics (thread 128)
+    uint32_t ntile = 0, nret = 0;  // tiles tested / retained by this CTA (also the stats)
     bool ok = true;
     uint8_t* dsrow_base = sdS + wg * 16384;  // this warpgroup's 64-column atom
     for (uint32_t k = 0; ok; ++k) {
@@ -460,12 +459,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           named_bar_sync(1, 256);  // every S^T load done before P overwrites it
         }
         if (*ast.flag) { ok = false; break; }
-        if (tid == 128) {
-          ++st_legal;
-          st_ret += keep ? 1u : 0u;
-          if (p.tile_mask)
-            p.tile_mask[((static_cast<size_t>(w.b) * p.H + h) * p.T + i) * p.T + w.j] = keep ? 1 : 0;
-        }
+        if (p.tile_mask && tid == 128)
+          p.tile_mask[((static_cast<size_t>(w.b) * p.H + h) * p.T + i) * p.T + w.j] = keep ? 1 : 0;
         if (!keep) {
           if (tid == 128) sh.dec = 0;
           tc_fence_before();
@@ -535,7 +530,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         warp_arrive(&sh.ds_full);
       }
     }
-    if (tid == 128) stats_add(p.stats, st_legal, st_ret, 0);
+    if (tid == 128) stats_add(p.stats, ntile, nret, 0);
   } else if (warp >= 12) {
     // ------------------------------------------------------------------ dQ drain + dK/dV epilogue
     const int wq = warp & 3;

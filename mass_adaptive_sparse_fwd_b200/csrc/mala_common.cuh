@@ -35,13 +35,14 @@ __device__ __forceinline__ void stats_add(unsigned long long* stats, uint32_t le
 #endif
 
 struct FwdParams {
-  int B, H, Hkv, L, T, G, npairs;
+  int B, H, Hkv, L, T, G, npairs;  // L, T: query rows and query blocks
+  int Lk, Tk, off;    // key rows and key blocks; query row q sits at position off + q
   int n_units;
   float scale_log2;   // scale * log2(e)
   float log2_tau;     // log2(tau); -inf when tau == 0
   void* O;            // [B, L, H, D] bf16
   float* LSE;         // [B, H, L]
-  uint8_t* tile_mask; // [B, H, T, T] or null
+  uint8_t* tile_mask; // [B, H, T, Tk] or null
   uint32_t* err;      // device error word
   uint32_t* sched;    // persistent scheduler counter (zeroed before launch)
   uint64_t budget_ns;

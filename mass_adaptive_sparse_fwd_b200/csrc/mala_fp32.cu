@@ -34,16 +34,20 @@ __device__ __forceinline__ float log_thr(float tau, int Lq, bool screen) {
   return logf(tau) - logf(static_cast<float>(Lq));
 }
 
-// Forward: one CTA per (b, h, query block i); K_j, V_j staged in shared memory.
+// Forward: one CTA per (b, h, query block i); K_j, V_j staged in shared memory.  The L
+// query rows are the last L of Lk key positions (row q at position off + q, off = Lk - L;
+// off = 0 for the ordinary forward, > 0 for a prefill chunk).
 __global__ void __launch_bounds__(kF32Threads)
     fp32_fwd_kernel(const float* __restrict__ Q, const float* __restrict__ K,
                     const float* __restrict__ V, float* __restrict__ O, float* __restrict__ LSE,
-                    int B, int H, int Hkv, int L, int d, float scale, float tau, bool screen,
-                    uint8_t* tile_mask, unsigned long long* stats) {
+                    int B, int H, int Hkv, int L, int Lk, int d, float scale, float tau,
+                    bool screen, uint8_t* tile_mask, unsigned long long* stats) {
   extern __shared__ float fsm[];
   float* sK = fsm;             // [128][d]
   float* sV = fsm + kTile * d;  // [128][d]
   const int T = (L + kTile - 1) / kTile;
+  const int Tk = (Lk + kTile - 1) / kTile;
+  const int off = Lk - L;
   const int i = blockIdx.x % T;
   const int h = (blockIdx.x / T) % H;
   const int b = blockIdx.x / (T * H);
@@ -51,27 +55,29 @@ __global__ void __launch_bounds__(kF32Threads)
   const int r = threadIdx.x;
   const int q = i * kTile + r;
   const bool valid = q < L;
+  const int pos = off + q;
   float qv[128], acc[128], s[kTile];
   for (int c = 0; c < d; ++c) {
     qv[c] = valid ? Q[((static_cast<size_t>(b) * L + q) * H + h) * d + c] : 0.f;
     acc[c] = 0.f;
   }
-  const float theta = log_thr(tau, q + 1, screen);
+  const float theta = log_thr(tau, pos + 1, screen);
   float m = -INFINITY, l = 0.f;
-  for (int j = i; j >= 0; --j) {  // diagonal first
+  const int j_last = (off + min(i * kTile + kTile - 1, L - 1)) / kTile;
+  for (int j = j_last; j >= 0; --j) {  // diagonal first
     __syncthreads();
     for (int e = r; e < kTile * d; e += kF32Threads) {
       const int k = j * kTile + e / d, c = e % d;
-      const size_t src = ((static_cast<size_t>(b) * L + k) * Hkv + g) * d + c;
-      sK[e] = k < L ? K[src] : 0.f;
-      sV[e] = k < L ? V[src] : 0.f;
+      const size_t src = ((static_cast<size_t>(b) * Lk + k) * Hkv + g) * d + c;
+      sK[e] = k < Lk ? K[src] : 0.f;
+      sV[e] = k < Lk ? V[src] : 0.f;
     }
     __syncthreads();
     float rmax = -INFINITY;
     bool has = false;
     for (int kk = 0; kk < kTile; ++kk) {
       const int k = j * kTile + kk;
-      const bool legal = valid && k <= q;
+      const bool legal = valid && k <= pos;
       s[kk] = legal ? scale * dot_rows(qv, sK + kk * d, d) : -INFINITY;
       if (legal) { has = true; rmax = fmaxf(rmax, s[kk]); }
     }
@@ -80,7 +86,7 @@ __global__ void __launch_bounds__(kF32Threads)
     const bool keep = __syncthreads_or(mine) != 0;
     if (r == 0) {
       stats_add(stats, 1, keep ? 1 : 0, 0);
-      if (tile_mask) tile_mask[((static_cast<size_t>(b) * H + h) * T + i) * T + j] = keep ? 1 : 0;
+      if (tile_mask) tile_mask[((static_cast<size_t>(b) * H + h) * T + i) * Tk + j] = keep ? 1 : 0;
     }
     if (!keep || !has) continue;
     const float mn = fmaxf(m, rmax);
@@ -350,7 +356,7 @@ cudaError_t set_smem(const void* fn, int bytes) {
 }  // namespace
 
 mala_status fp32_fwd(const float* Q, const float* K, const float* V, float* O, float* LSE, int B,
-                     int H, int Hkv, int L, int d, float scale, float tau, bool screen,
+                     int H, int Hkv, int L, int Lk, int d, float scale, float tau, bool screen,
                      uint8_t* ws, uint8_t* tile_mask, cudaStream_t stream) {
   const int T = (L + kTile - 1) / kTile;
   const int smem = 2 * kTile * d * static_cast<int>(sizeof(float));
@@ -358,8 +364,8 @@ mala_status fp32_fwd(const float* Q, const float* K, const float* V, float* O, f
       ws ? reinterpret_cast<unsigned long long*>(ws + kStatsOffset) : nullptr;
   if (set_smem(reinterpret_cast<const void*>(fp32_fwd_kernel), smem) != cudaSuccess)
     return MALA_ERR_CUDA;
-  fp32_fwd_kernel<<<B * H * T, kF32Threads, smem, stream>>>(Q, K, V, O, LSE, B, H, Hkv, L, d,
-                                                            scale, tau, screen, tile_mask, stats);
+  fp32_fwd_kernel<<<B * H * T, kF32Threads, smem, stream>>>(
+      Q, K, V, O, LSE, B, H, Hkv, L, Lk, d, scale, tau, screen, tile_mask, stats);
   return cudaGetLastError() == cudaSuccess ? MALA_OK : MALA_ERR_CUDA;
 }
 

@@ -6,7 +6,11 @@
 // One persistent CTA per SM pulls work units from an atomic counter.  A unit is one
 // 128-row query block i of two query heads that share a KV head (two "slots"), so both
 // slots stream the same K_j / V_j tiles; units are numbered heaviest first (largest i).
-// Within a unit the key blocks are visited j = i, i-1, ..., 0 (diagonal first).
+// Within a unit the key blocks are visited from the block of the unit's last query
+// position down to 0 (diagonal first).  For chunked prefill (§2.3: the forward serves
+// inference prefill) the L query rows are the last L of Lk key positions: row q sits at
+// position off + q, off = Lk - L, attends to keys <= its position and has L_q = off + q + 1;
+// with off = 0 this is the ordinary causal forward.
 //
 // Warp roles (384 threads):
 //   warp 0      TMA producer: Q of both slots, then K_j and V_j per key block into a
@@ -21,7 +25,7 @@
 // Retention test (Eq. 3) per row q in the log2 domain: with the running state
 // (m, l) of retained tiles, log2 Z = m + log2 l.  A row keeps the tile if l == 0
 // (its first legal tile) or rowmax(S) * scale * log2(e) >= m + log2(l) + log2(tau/L_q),
-// L_q = q + 1; rows with no legal key in the tile (above the diagonal, or q >= L) do
+// L_q = position + 1; rows with no legal key in the tile (above the diagonal, or q >= L) do
 // not vote.  The tile is retained if any row keeps it (bar.red.or over the 128
 // threads).  A skipped tile leaves m, l and O untouched and costs only the QK^T MMA,
 // the TMEM load of S and the row maxima: no exponentials, no P store, no PV MMA.
@@ -76,6 +80,12 @@ struct Unit {
   int b, g, i, h0;
   bool active[2];
 };
+
+// Last key block holding a legal key of query block i (its last row's position).
+__device__ __forceinline__ int last_key_tile(const FwdParams& p, int i) {
+  const int q_last = min(i * kTile + kTile - 1, p.L - 1);
+  return (p.off + q_last) / kTile;
+}
 
 __device__ __forceinline__ Unit decode_unit(const FwdParams& p, int u) {
   const int nbg = p.B * p.Hkv * p.npairs;
@@ -166,8 +176,9 @@ __global__ void __launch_bounds__(384, 1)
                         w.h0 + s, w.i * kTile, w.b);
           ++nq[s];
         }
-        for (int t = 0; t <= w.i && ok; ++t, ++c) {
-          const int j = w.i - t;
+        const int jl = last_key_tile(p, w.i);
+        for (int t = 0; t <= jl && ok; ++t, ++c) {
+          const int j = jl - t;
           const int st = c % NS;
           if (c >= NS && !(ok = mbar_wait(&sh.kv_empty[st], ((c / NS) - 1) & 1, ast, 3))) break;
           mbar_arrive_expect_tx(&sh.k_full[st], C::TILE_BYTES);
@@ -228,7 +239,7 @@ __global__ void __launch_bounds__(384, 1)
         }
         if (!ok) break;
         bool o_started[2] = {false, false};
-        const int n = w.i + 1;
+        const int n = last_key_tile(p, w.i) + 1;
         // prologue: S for the diagonal tile
         {
           const int st = c % NS;
@@ -291,8 +302,7 @@ __global__ void __launch_bounds__(384, 1)
     const uint32_t tS = tb + s * 128 + lane_off;
     const uint32_t tO = tb + 256 + s * D + lane_off;
     const float NEG_INF = -INFINITY;
-    uint32_t ns = 0, npv = 0;
-    uint32_t st_legal = 0, st_ret = 0;  // call statistics (row-0 thread of the slot)
+    uint32_t ns = 0, npv = 0;  // tiles tested / retained by this slot (also the stats)
     bool ok = true;
     for (uint32_t k = 0; ok; ++k) {
       const int ring = k & 1;
@@ -308,23 +318,29 @@ __global__ void __launch_bounds__(384, 1)
       const int h = w.h0 + s;
       const int q = w.i * kTile + r;
       const bool valid = q < p.L;
-      const float thr2 = kScreen ? (p.log2_tau - __log2f(static_cast<float>(q + 1))) : NEG_INF;
+      // L_q = position + 1 (the position is q in a full forward, off + q in a chunk)
+      const float thr2 =
+          kScreen ? (p.log2_tau - __log2f(static_cast<float>(p.off + q + 1))) : NEG_INF;
       float m2 = NEG_INF, l = 0.f;
       const uint32_t npv_unit0 = npv;
-      const int n = w.i + 1;
+      const int jl = last_key_tile(p, w.i);
+      const int pos0 = p.off + w.i * kTile;  // position of the block's first row
+      const int n = jl + 1;
       for (int t = 0; t < n; ++t) {
-        const int j = w.i - t;
+        const int j = jl - t;
         // A failed wait never leaves the loop before the next named barrier of the
         // warpgroup: the abort flag is set and checked right after the vote.
         const bool got = mbar_wait(&sh.s_full[s], ns & 1, ast, 21);
         ++ns;
         tc_fence_after();
         // pass 1: row maximum of the raw scores (the scale is positive, so it commutes
-        // with max), 64 columns at a time; only the diagonal tile and rows past the end
-        // need masking (keys c <= r are legal on the diagonal)
+        // with max), 64 columns at a time; only tiles that reach past the block's first
+        // position (the diagonal tile, and its neighbour when the chunk offset is not a
+        // multiple of 128) and rows past the end need masking: key c is legal for row r
+        // iff c <= lim = position - 128 j
         const bool warp_ok = __all_sync(0xffffffffu, got);
-        const bool masked = (t == 0) || !valid;
-        const int lim = valid ? r : -1;
+        const bool masked = (j * kTile + kTile - 1 > pos0) || !valid;
+        const int lim = valid ? (pos0 + r - j * kTile) : -1;
         float rraw = NEG_INF;
         if (warp_ok) {
 #pragma unroll
@@ -356,12 +372,8 @@ __global__ void __launch_bounds__(384, 1)
           keep = named_bar_or(1 + s, 128, mine);
           if (*ast.flag) { ok = false; break; }
         }
-        if (r == 0) {
-          ++st_legal;
-          st_ret += keep ? 1u : 0u;
-          if (p.tile_mask)
-            p.tile_mask[((static_cast<size_t>(w.b) * p.H + h) * p.T + w.i) * p.T + j] = keep ? 1 : 0;
-        }
+        if (p.tile_mask && r == 0)
+          p.tile_mask[((static_cast<size_t>(w.b) * p.H + h) * p.T + w.i) * p.Tk + j] = keep ? 1 : 0;
         if (!keep) {
           if (r == 0) sh.dec[s] = 0;
           tc_fence_before();
@@ -454,7 +466,7 @@ __global__ void __launch_bounds__(384, 1)
       if (valid) p.LSE[(static_cast<size_t>(w.b) * p.H + h) * p.L + q] = (m2 + __log2f(l)) * kLn2;
       tc_fence_before();
     }
-    if (r == 0) stats_add(p.stats, st_legal, st_ret, 0);
+    if (r == 0) stats_add(p.stats, ns, npv, 0);
   }
 
   tc_fence_before();

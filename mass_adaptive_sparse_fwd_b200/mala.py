@@ -24,7 +24,8 @@ MALA_BF16, MALA_FP32 = 0, 1
 MALA_FLAG_ALWAYS_TEST = 1
 TILE = 128
 
-EXPORTED = ("mala_fwd", "mala_bwd", "mala_decode", "mala_decode_noalloc", "mala_get_stats",
+EXPORTED = ("mala_fwd", "mala_fwd_prefill", "mala_bwd", "mala_decode", "mala_decode_noalloc",
+            "mala_get_stats",
             "mala_fwd_workspace_bytes",
             "mala_bwd_workspace_bytes", "mala_decode_workspace_bytes", "mala_decode_num_splits",
             "mala_read_device_error", "mala_set_wait_budget_ns", "mala_status_string",
@@ -50,6 +51,8 @@ def load_library(path: str = _LIB_PATH) -> ctypes.CDLL:
     vp, ci, cf, cu, sz = (ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_uint,
                           ctypes.c_size_t)
     lib.mala_fwd.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, cf, cf, cu, vp, sz, vp, vp]
+    lib.mala_fwd_prefill.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, ci, cf, cf, cu,
+                                     vp, sz, vp, vp]
     lib.mala_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, cf, cf,
                              cu, vp, sz, vp, vp]
     lib.mala_decode.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, cf, cf, ci, cu, vp, sz,
@@ -57,7 +60,7 @@ def load_library(path: str = _LIB_PATH) -> ctypes.CDLL:
     lib.mala_decode_noalloc.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, cf, cf, ci, cu,
                                         vp, vp]
     lib.mala_decode_noalloc.restype = ci
-    for f in ("mala_fwd", "mala_bwd", "mala_decode", "mala_read_device_error",
+    for f in ("mala_fwd", "mala_fwd_prefill", "mala_bwd", "mala_decode", "mala_read_device_error",
               "mala_set_wait_budget_ns"):
         getattr(lib, f).restype = ci
     lib.mala_fwd_workspace_bytes.argtypes = [ci] * 6
@@ -147,6 +150,25 @@ def mala_fwd(Q, K, V, scale, tau, O=None, LSE=None, flags=0, workspace=None, til
                        _dtype_code(Q), float(scale), float(tau), flags, _ptr(workspace), ws_bytes,
                        _ptr(tile_mask), _stream(stream))
     _check("mala_fwd", st)
+    return O, LSE
+
+
+def mala_fwd_prefill(Q, K, V, scale, tau, O=None, LSE=None, flags=0, workspace=None,
+                     tile_mask=None, stream=None):
+    """Forward of a prefill chunk through the C ABI: Q [B,N_q,H,d] are the last N_q
+    positions of the sequence whose keys K/V [B,N_k,H_kv,d] (N_k >= N_q) include them.
+    Returns (O [B,N_q,H,d], LSE [B,H,N_q])."""
+    B, Nq, H, d = Q.shape
+    Nk, H_kv = K.shape[1], K.shape[2]
+    if O is None:
+        O = torch.empty_like(Q)
+    if LSE is None:
+        LSE = torch.empty((B, H, Nq), dtype=torch.float32, device=Q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel()
+    st = _lib.mala_fwd_prefill(_ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(LSE), B, H, H_kv, Nq, Nk,
+                               d, _dtype_code(Q), float(scale), float(tau), flags,
+                               _ptr(workspace), ws_bytes, _ptr(tile_mask), _stream(stream))
+    _check("mala_fwd_prefill", st)
     return O, LSE
 
 
