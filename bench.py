@@ -552,6 +552,49 @@ def run_mala(args, dist: Dist):
             "tau1_gbs": hb1 / (hd1 * 1e-6) / 1e9, "tau0_gbs": hb0 / (hd0 * 1e-6) / 1e9}
         del hq, hK, hV, hO, hL, hws
 
+    # chunked prefill: the last 4096 queries of the 32K sink + band sequence against all
+    # 32768 keys (causal offset 28672), tau = 1 and tau = 0
+    prefill = None
+    if not args.no_skip_regime:
+        wp = rank_workload(synth.WORKLOADS[TRAIN], dist.rank)
+        loc = synth.make_training(wp)
+        Nq, Nk = 4096, wp.L
+        pQ = bf(np.ascontiguousarray(loc["Q"][:, Nk - Nq:]))
+        pK, pV = bf(loc["K"]), bf(loc["V"])
+        del loc
+        pO = torch.empty_like(pQ)
+        pL = torch.empty((wp.B, wp.H, Nq), dtype=torch.float32, device=dev)
+        pws = mala.alloc_workspace(mala.fwd_workspace_bytes(wp.B, wp.H, wp.H_kv, Nq, wp.d), dev)
+
+        def ptime(tau):
+            for _ in range(args.warmup):
+                mala.mala_fwd_prefill(pQ, pK, pV, wp.scale, tau, O=pO, LSE=pL, workspace=pws)
+            torch.cuda.synchronize(dev)
+            dist.barrier()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(args.steps):
+                mala.mala_fwd_prefill(pQ, pK, pV, wp.scale, tau, O=pO, LSE=pL, workspace=pws)
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            dist.barrier()
+            st = mala.get_stats(pws)  # the last timed call's tile counts
+            return dist.max(e0.elapsed_time(e1) / args.steps, device=dev), st
+
+        pt1, pst = ptime(TAU)
+        pt0, _ = ptime(0.0)
+        per_tile = 2.0 * wp.d * 128 * 128
+        fl1 = per_tile * (pst["legal_tiles"] + pst["retained_tiles"])
+        fl0 = per_tile * 2 * pst["legal_tiles"]
+        prefill = {"workload": f"last {Nq} queries of {TRAIN} against its {Nk} keys "
+                               f"(B={wp.B},H={wp.H},H_kv={wp.H_kv},d={wp.d}; offset {Nk - Nq})",
+                   "legal_tiles": pst["legal_tiles"],
+                   "retained": pst["retained_tiles"] / max(pst["legal_tiles"], 1),
+                   "tau1_ms": pt1, "tau0_ms": pt0, "speedup_vs_tau0": pt0 / pt1,
+                   "tau1_executed_tflops": fl1 / (pt1 * 1e-3) / 1e12,
+                   "tau0_tflops": fl0 / (pt0 * 1e-3) / 1e12}
+        del pQ, pK, pV, pO, pL, pws
+
     cpu = None
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
         ms, spent, desc = oracle_sample(wt, wd, train, dec, S)
@@ -602,6 +645,7 @@ def run_mala(args, dist: Dist):
             "e2e": e2e,
             "cpu_baseline": cpu,
             "skip_regime": skip,
+            "prefill": prefill,
         }
         print(json.dumps(line), flush=True)
 
