@@ -96,6 +96,31 @@ mala_status mala_fwd_prefill(const void* Q, const void* K, const void* V, void* 
                              size_t workspace_bytes, uint8_t* tile_mask, void* stream);
 
 /*
+ * mala_fwd_varlen - MALA forward of a packed batch of sequences of different lengths.
+ * "MassAlloc Attention", §2.3 (the forward serves inference prefill) with the rules of
+ * mala_fwd_prefill applied to each sequence on its own.
+ *   Sequence s owns query rows [cu_seqlens_q[s], cu_seqlens_q[s+1]) of Q / O and key
+ *   rows [cu_seqlens_k[s], cu_seqlens_k[s+1]) of K / V; its N_q,s queries are the last
+ *   N_q,s of its N_k,s >= N_q,s positions (N_q,s == N_k,s: a full causal sequence; a
+ *   sequence may have N_q,s == 0).
+ *   Q, O [total_q, H, d]; K, V [total_k, H_kv, d] (bf16, d in {64, 128}); LSE [H, total_q]
+ *   float32.  cu_seqlens_q / cu_seqlens_k are HOST arrays of n_seqs + 1 non-decreasing
+ *   offsets starting at 0.
+ *   The workspace is required (mala_fwd_varlen_workspace_bytes): it receives a table of
+ *   the batch's (sequence, query block) units, heaviest first, copied from host memory
+ *   with cudaMemcpyAsync, so the call waits for earlier work on `stream` before it
+ *   returns (pageable staging) and cannot be captured in a CUDA graph.  No tile_mask;
+ *   mala_get_stats reports the call's tiles.  Each sequence's results equal those of
+ *   mala_fwd_prefill on that sequence alone.
+ */
+size_t mala_fwd_varlen_workspace_bytes(const int* cu_seqlens_q, int n_seqs, int H, int H_kv,
+                                       int d, int dtype);
+mala_status mala_fwd_varlen(const void* Q, const void* K, const void* V, void* O, float* LSE,
+                            const int* cu_seqlens_q, const int* cu_seqlens_k, int n_seqs, int H,
+                            int H_kv, int d, int dtype, float scale, float tau, unsigned flags,
+                            void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * mala_bwd - MALA backward.
  * "MassAlloc Attention", §2.2 (offline sparse probability, Eq. (4)), App. A
  * Algorithm 2 and A.1 (fused backward execution).  O and LSE are the forward's

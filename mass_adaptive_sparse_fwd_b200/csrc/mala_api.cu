@@ -4,7 +4,9 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
+#include <vector>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
@@ -222,6 +224,8 @@ mala_status run_fwd(const void* Q, const void* K, const void* V, void* O, float*
     FwdParams p;
     p.B = B; p.H = H; p.Hkv = H_kv; p.L = L; p.T = T; p.G = H / H_kv;
     p.Lk = Lk; p.Tk = Tk; p.off = Lk - L;
+    p.Lrows = L;
+    p.vtab = nullptr;
     p.npairs = (p.G + 1) / 2;
     p.n_units = T * B * H_kv * p.npairs;
     p.scale_log2 = scale * kLog2e;
@@ -248,6 +252,92 @@ mala_status mala_fwd(const void* Q, const void* K, const void* V, void* O, float
                      uint8_t* tile_mask, void* stream) {
   return run_fwd(Q, K, V, O, LSE, B, H, H_kv, L, L, d, dtype, scale, tau, flags, workspace,
                  workspace_bytes, tile_mask, stream);
+}
+
+size_t mala_fwd_varlen_workspace_bytes(const int* cu_seqlens_q, int n_seqs, int H, int H_kv,
+                                       int d, int dtype) {
+  if (!cu_seqlens_q || n_seqs <= 0 || H <= 0 || H_kv <= 0 || H % H_kv || dtype != MALA_BF16 ||
+      (d != 64 && d != 128))
+    return 0;
+  long long blocks = 0;
+  for (int s = 0; s < n_seqs; ++s) {
+    const int Lq = cu_seqlens_q[s + 1] - cu_seqlens_q[s];
+    if (Lq < 0) return 0;
+    blocks += (Lq + kTile - 1) / kTile;
+  }
+  return kWorkspaceHeader + static_cast<size_t>(blocks) * sizeof(VarlenBlock);
+}
+
+mala_status mala_fwd_varlen(const void* Q, const void* K, const void* V, void* O, float* LSE,
+                            const int* cu_seqlens_q, const int* cu_seqlens_k, int n_seqs, int H,
+                            int H_kv, int d, int dtype, float scale, float tau, unsigned flags,
+                            void* workspace, size_t workspace_bytes, void* stream) {
+  if (!cu_seqlens_q || !cu_seqlens_k || n_seqs <= 0) return MALA_ERR_INVALID_ARG;
+  if (cu_seqlens_q[0] != 0 || cu_seqlens_k[0] != 0) return MALA_ERR_INVALID_ARG;
+  std::vector<VarlenBlock> tab;
+  for (int s = 0; s < n_seqs; ++s) {
+    const int Lq = cu_seqlens_q[s + 1] - cu_seqlens_q[s];
+    const int Lk = cu_seqlens_k[s + 1] - cu_seqlens_k[s];
+    if (Lq < 0 || Lk < Lq) return MALA_ERR_INVALID_ARG;
+    for (int i = 0; i < (Lq + kTile - 1) / kTile; ++i) {
+      VarlenBlock e{};
+      e.qrow0 = cu_seqlens_q[s];
+      e.krow0 = cu_seqlens_k[s];
+      e.L = Lq;
+      e.off = Lk - Lq;
+      e.i = i;
+      tab.push_back(e);
+    }
+  }
+  const int total_q = cu_seqlens_q[n_seqs], total_k = cu_seqlens_k[n_seqs];
+  if (tab.empty()) return MALA_OK;  // no query rows: nothing to do
+  if (!common_args_ok(1, H, H_kv, total_q, d, dtype, scale, tau)) return MALA_ERR_INVALID_ARG;
+  if (dtype != MALA_BF16) return MALA_ERR_UNSUPPORTED;  // packed batches: tensor-core path only
+  if (d != 64 && d != 128) return MALA_ERR_UNSUPPORTED;
+  if (!Q || !K || !V || !O || !LSE || !workspace) return MALA_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(workspace))
+    return MALA_ERR_INVALID_ARG;
+  const size_t need = mala_fwd_varlen_workspace_bytes(cu_seqlens_q, n_seqs, H, H_kv, d, dtype);
+  if (workspace_bytes < need) return MALA_ERR_WORKSPACE;
+  // heaviest first: the blocks with the most key tiles
+  auto weight = [](const VarlenBlock& e) {
+    return (e.off + std::min(e.i * kTile + kTile - 1, e.L - 1)) / kTile + 1;
+  };
+  std::stable_sort(tab.begin(), tab.end(), [&](const VarlenBlock& a, const VarlenBlock& b) {
+    return weight(a) > weight(b);
+  });
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const bool screen = (tau > 0.f) || (flags & MALA_FLAG_ALWAYS_TEST);
+  CUtensorMap tq, tk, tv;
+  if (!make_tile_map(&tq, Q, d, H, total_q, 1) || !make_tile_map(&tk, K, d, H_kv, total_k, 1) ||
+      !make_tile_map(&tv, V, d, H_kv, total_k, 1))
+    return MALA_ERR_CUDA;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  uint32_t* hdr = reinterpret_cast<uint32_t*>(ws);
+  VarlenBlock* dtab = reinterpret_cast<VarlenBlock*>(ws + kWorkspaceHeader);
+  // the table comes from pageable host memory: the copy is staged before the call returns
+  if (cudaMemcpyAsync(dtab, tab.data(), tab.size() * sizeof(VarlenBlock), cudaMemcpyHostToDevice,
+                      st) != cudaSuccess ||
+      cudaMemsetAsync(hdr + kHdrSched0, 0, 3 * sizeof(uint32_t), st) != cudaSuccess ||
+      cudaMemsetAsync(ws + kStatsOffset, 0, 3 * sizeof(unsigned long long), st) != cudaSuccess)
+    return MALA_ERR_CUDA;
+  FwdParams p;
+  p.B = 1; p.H = H; p.Hkv = H_kv; p.G = H / H_kv;
+  p.L = total_q; p.T = 0; p.Lk = total_k; p.Tk = 0; p.off = 0;
+  p.Lrows = total_q;
+  p.vtab = dtab;
+  p.npairs = (p.G + 1) / 2;
+  p.n_units = static_cast<int>(tab.size()) * H_kv * p.npairs;
+  p.scale_log2 = scale * kLog2e;
+  p.log2_tau = (tau > 0.f) ? std::log2(tau) : -INFINITY;
+  p.O = O; p.LSE = LSE; p.tile_mask = nullptr;
+  p.err = hdr + kHdrError;
+  p.sched = hdr + kHdrSched0;
+  p.budget_ns = wait_budget_ns();
+  p.stats = reinterpret_cast<unsigned long long*>(ws + kStatsOffset);
+  const int grid = p.n_units < sm_count() ? p.n_units : sm_count();
+  return launch_fwd_bf16(tq, tk, tv, p, d, screen, grid, st) == cudaSuccess ? MALA_OK
+                                                                            : MALA_ERR_CUDA;
 }
 
 mala_status mala_fwd_prefill(const void* Q, const void* K, const void* V, void* O, float* LSE,

@@ -34,9 +34,20 @@ __device__ __forceinline__ void stats_add(unsigned long long* stats, uint32_t le
 }
 #endif
 
+// One query block of one sequence of a packed (varlen) batch, in the order the
+// persistent CTAs take them (heaviest first).
+struct VarlenBlock {
+  int qrow0, krow0;  // packed row of the sequence's first query / first key
+  int L, off;        // the sequence's query rows and causal offset (key rows - L)
+  int i;             // query block within the sequence
+  int pad[3];
+};
+
 struct FwdParams {
   int B, H, Hkv, L, T, G, npairs;  // L, T: query rows and query blocks
   int Lk, Tk, off;    // key rows and key blocks; query row q sits at position off + q
+  int Lrows;          // rows of Q / O per batch entry (L; the packed total for varlen)
+  const VarlenBlock* vtab;  // varlen: one entry per (sequence, query block), else null
   int n_units;
   float scale_log2;   // scale * log2(e)
   float log2_tau;     // log2(tau); -inf when tau == 0

@@ -79,22 +79,43 @@ static_assert(FwdCfg<64>::SMEM + sizeof(FwdShared) <= 232448, "forward smem budg
 struct Unit {
   int b, g, i, h0;
   bool active[2];
+  int qrow0, krow0;  // first row of the sequence in Q / K (packed varlen batch), else 0
+  int L, off;        // the sequence's query rows and causal offset
 };
 
-// Last key block holding a legal key of query block i (its last row's position).
-__device__ __forceinline__ int last_key_tile(const FwdParams& p, int i) {
-  const int q_last = min(i * kTile + kTile - 1, p.L - 1);
-  return (p.off + q_last) / kTile;
+// Last key block holding a legal key of the unit's query block (its last row's position).
+__device__ __forceinline__ int last_key_tile(const Unit& w) {
+  const int q_last = min(w.i * kTile + kTile - 1, w.L - 1);
+  return (w.off + q_last) / kTile;
 }
 
 __device__ __forceinline__ Unit decode_unit(const FwdParams& p, int u) {
-  const int nbg = p.B * p.Hkv * p.npairs;
   Unit w;
-  w.i = p.T - 1 - u / nbg;
-  const int r = u % nbg;
-  w.b = r / (p.Hkv * p.npairs);
-  w.g = (r / p.npairs) % p.Hkv;
-  const int hp = r % p.npairs;
+  int r, hp;
+  if (p.vtab) {  // packed batch: the table lists (sequence, query block), heaviest first
+    const int nbg = p.Hkv * p.npairs;
+    const VarlenBlock e = p.vtab[u / nbg];
+    r = u % nbg;
+    w.b = 0;
+    w.g = r / p.npairs;
+    hp = r % p.npairs;
+    w.i = e.i;
+    w.qrow0 = e.qrow0;
+    w.krow0 = e.krow0;
+    w.L = e.L;
+    w.off = e.off;
+  } else {
+    const int nbg = p.B * p.Hkv * p.npairs;
+    w.i = p.T - 1 - u / nbg;
+    r = u % nbg;
+    w.b = r / (p.Hkv * p.npairs);
+    w.g = (r / p.npairs) % p.Hkv;
+    hp = r % p.npairs;
+    w.qrow0 = 0;
+    w.krow0 = 0;
+    w.L = p.L;
+    w.off = p.off;
+  }
   w.h0 = w.g * p.G + 2 * hp;
   w.active[0] = true;
   w.active[1] = (2 * hp + 1) < p.G;
@@ -173,10 +194,10 @@ __global__ void __launch_bounds__(384, 1)
           mbar_arrive_expect_tx(&sh.q_full[s], C::TILE_BYTES);
           for (int x = 0; x < C::BOXES; ++x)
             tma_load_4d(sQ + s * C::TILE_BYTES + x * 16384, &tmQ, &sh.q_full[s], x * 64,
-                        w.h0 + s, w.i * kTile, w.b);
+                        w.h0 + s, w.qrow0 + w.i * kTile, w.b);
           ++nq[s];
         }
-        const int jl = last_key_tile(p, w.i);
+        const int jl = last_key_tile(w);
         for (int t = 0; t <= jl && ok; ++t, ++c) {
           const int j = jl - t;
           const int st = c % NS;
@@ -184,11 +205,11 @@ __global__ void __launch_bounds__(384, 1)
           mbar_arrive_expect_tx(&sh.k_full[st], C::TILE_BYTES);
           for (int x = 0; x < C::BOXES; ++x)
             tma_load_4d(sK + st * C::TILE_BYTES + x * 16384, &tmK, &sh.k_full[st], x * 64, w.g,
-                        j * kTile, w.b);
+                        w.krow0 + j * kTile, w.b);
           mbar_arrive_expect_tx(&sh.v_full[st], C::TILE_BYTES);
           for (int x = 0; x < C::BOXES; ++x)
             tma_load_4d(sV + st * C::TILE_BYTES + x * 16384, &tmV, &sh.v_full[st], x * 64, w.g,
-                        j * kTile, w.b);
+                        w.krow0 + j * kTile, w.b);
         }
       }
       if (!ok) {
@@ -239,7 +260,7 @@ __global__ void __launch_bounds__(384, 1)
         }
         if (!ok) break;
         bool o_started[2] = {false, false};
-        const int n = last_key_tile(p, w.i) + 1;
+        const int n = last_key_tile(w) + 1;
         // prologue: S for the diagonal tile
         {
           const int st = c % NS;
@@ -317,14 +338,14 @@ __global__ void __launch_bounds__(384, 1)
       if (!w.active[s]) continue;
       const int h = w.h0 + s;
       const int q = w.i * kTile + r;
-      const bool valid = q < p.L;
+      const bool valid = q < w.L;
       // L_q = position + 1 (the position is q in a full forward, off + q in a chunk)
       const float thr2 =
-          kScreen ? (p.log2_tau - __log2f(static_cast<float>(p.off + q + 1))) : NEG_INF;
+          kScreen ? (p.log2_tau - __log2f(static_cast<float>(w.off + q + 1))) : NEG_INF;
       float m2 = NEG_INF, l = 0.f;
       const uint32_t npv_unit0 = npv;
-      const int jl = last_key_tile(p, w.i);
-      const int pos0 = p.off + w.i * kTile;  // position of the block's first row
+      const int jl = last_key_tile(w);
+      const int pos0 = w.off + w.i * kTile;  // position of the block's first row
       const int n = jl + 1;
       for (int t = 0; t < n; ++t) {
         const int j = jl - t;
@@ -445,7 +466,7 @@ __global__ void __launch_bounds__(384, 1)
       tc_fence_after();
       const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
       __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.O) +
-                            ((static_cast<size_t>(w.b) * p.L + q) * p.H + h) * D;
+                            ((static_cast<size_t>(w.b) * p.Lrows + w.qrow0 + q) * p.H + h) * D;
 #pragma unroll
       for (int cc = 0; cc < D / 32; ++cc) {
         uint32_t o[32];
@@ -463,7 +484,8 @@ __global__ void __launch_bounds__(384, 1)
           }
         }
       }
-      if (valid) p.LSE[(static_cast<size_t>(w.b) * p.H + h) * p.L + q] = (m2 + __log2f(l)) * kLn2;
+      if (valid)
+        p.LSE[(static_cast<size_t>(w.b) * p.H + h) * p.Lrows + w.qrow0 + q] = (m2 + __log2f(l)) * kLn2;
       tc_fence_before();
     }
     if (r == 0) stats_add(p.stats, ns, npv, 0);

@@ -24,8 +24,8 @@ MALA_BF16, MALA_FP32 = 0, 1
 MALA_FLAG_ALWAYS_TEST = 1
 TILE = 128
 
-EXPORTED = ("mala_fwd", "mala_fwd_prefill", "mala_bwd", "mala_decode", "mala_decode_noalloc",
-            "mala_get_stats",
+EXPORTED = ("mala_fwd", "mala_fwd_prefill", "mala_fwd_varlen", "mala_bwd", "mala_decode",
+            "mala_decode_noalloc", "mala_get_stats", "mala_fwd_varlen_workspace_bytes",
             "mala_fwd_workspace_bytes",
             "mala_bwd_workspace_bytes", "mala_decode_workspace_bytes", "mala_decode_num_splits",
             "mala_read_device_error", "mala_set_wait_budget_ns", "mala_status_string",
@@ -53,6 +53,11 @@ def load_library(path: str = _LIB_PATH) -> ctypes.CDLL:
     lib.mala_fwd.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, cf, cf, cu, vp, sz, vp, vp]
     lib.mala_fwd_prefill.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, ci, cf, cf, cu,
                                      vp, sz, vp, vp]
+    ip = ctypes.POINTER(ctypes.c_int)
+    lib.mala_fwd_varlen.argtypes = [vp, vp, vp, vp, vp, ip, ip, ci, ci, ci, ci, ci, cf, cf, cu,
+                                    vp, sz, vp]
+    lib.mala_fwd_varlen_workspace_bytes.argtypes = [ip, ci, ci, ci, ci, ci]
+    lib.mala_fwd_varlen_workspace_bytes.restype = sz
     lib.mala_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, cf, cf,
                              cu, vp, sz, vp, vp]
     lib.mala_decode.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, cf, cf, ci, cu, vp, sz,
@@ -60,7 +65,8 @@ def load_library(path: str = _LIB_PATH) -> ctypes.CDLL:
     lib.mala_decode_noalloc.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, cf, cf, ci, cu,
                                         vp, vp]
     lib.mala_decode_noalloc.restype = ci
-    for f in ("mala_fwd", "mala_fwd_prefill", "mala_bwd", "mala_decode", "mala_read_device_error",
+    for f in ("mala_fwd", "mala_fwd_prefill", "mala_fwd_varlen", "mala_bwd", "mala_decode",
+              "mala_read_device_error",
               "mala_set_wait_budget_ns"):
         getattr(lib, f).restype = ci
     lib.mala_fwd_workspace_bytes.argtypes = [ci] * 6
@@ -169,6 +175,38 @@ def mala_fwd_prefill(Q, K, V, scale, tau, O=None, LSE=None, flags=0, workspace=N
                                d, _dtype_code(Q), float(scale), float(tau), flags,
                                _ptr(workspace), ws_bytes, _ptr(tile_mask), _stream(stream))
     _check("mala_fwd_prefill", st)
+    return O, LSE
+
+
+def _int_array(xs):
+    xs = [int(x) for x in xs]
+    return (ctypes.c_int * len(xs))(*xs)
+
+
+def varlen_workspace_bytes(cu_seqlens_q, H, H_kv, d, dtype=MALA_BF16) -> int:
+    return _lib.mala_fwd_varlen_workspace_bytes(_int_array(cu_seqlens_q), len(cu_seqlens_q) - 1,
+                                                H, H_kv, d, dtype)
+
+
+def mala_fwd_varlen(Q, K, V, cu_seqlens_q, cu_seqlens_k, scale, tau, O=None, LSE=None, flags=0,
+                    workspace=None, stream=None):
+    """Forward of a packed batch through the C ABI: Q [total_q,H,d], K/V [total_k,H_kv,d];
+    cu_seqlens_* are host sequences of n+1 offsets.  Returns (O [total_q,H,d],
+    LSE [H,total_q])."""
+    total_q, H, d = Q.shape
+    H_kv = K.shape[1]
+    n = len(cu_seqlens_q) - 1
+    if O is None:
+        O = torch.empty_like(Q)
+    if LSE is None:
+        LSE = torch.empty((H, total_q), dtype=torch.float32, device=Q.device)
+    if workspace is None:
+        workspace = alloc_workspace(varlen_workspace_bytes(cu_seqlens_q, H, H_kv, d), Q.device)
+    st = _lib.mala_fwd_varlen(_ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(LSE),
+                              _int_array(cu_seqlens_q), _int_array(cu_seqlens_k), n, H, H_kv, d,
+                              _dtype_code(Q), float(scale), float(tau), flags, _ptr(workspace),
+                              workspace.numel(), _stream(stream))
+    _check("mala_fwd_varlen", st)
     return O, LSE
 
 

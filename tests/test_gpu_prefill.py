@@ -152,3 +152,74 @@ def test_prefill_4k_chunk_of_32k_sampled(orc, mala):
     Qc = np.ascontiguousarray(inp["Q"][:, Nk - Nq:])
     units = [(0, 0, 31), (0, 17, 0), (0, 31, 15)]
     check_prefill(orc, mala, w0, Qc, inp["K"], inp["V"], 1.0, units=units)
+
+
+# ---------------------------------------------------------------------------- packed batches
+
+
+def _packed(seqs, H, Hkv, d, structure="peaked"):
+    """seqs: list of (N_q, N_k).  Returns per-sequence (Qc, K, V) and the packed arrays."""
+    parts = []
+    for s, (nq, nk) in enumerate(seqs):
+        if nk == 0:
+            parts.append((np.zeros((1, 0, H, d), np.float32), np.zeros((1, 0, Hkv, d), np.float32),
+                          np.zeros((1, 0, Hkv, d), np.float32), None))
+            continue
+        w, Qc, K, V, _ = chunk(1, H, Hkv, nq, nk, d, structure, seed=70 + s)
+        parts.append((Qc, K, V, w))
+    cu_q = np.concatenate([[0], np.cumsum([p[0].shape[1] for p in parts])]).astype(int)
+    cu_k = np.concatenate([[0], np.cumsum([p[1].shape[1] for p in parts])]).astype(int)
+    Qp = np.concatenate([p[0][0] for p in parts], axis=0)
+    Kp = np.concatenate([p[1][0] for p in parts], axis=0)
+    Vp = np.concatenate([p[2][0] for p in parts], axis=0)
+    return parts, cu_q, cu_k, Qp, Kp, Vp
+
+
+@pytest.mark.parametrize("tau", [0.0, 1.0])
+def test_varlen_equals_per_sequence_prefill_bitwise(mala, tau):
+    H, Hkv, d = 4, 2, 128
+    seqs = [(300, 777), (128, 128), (1, 513), (0, 50), (517, 517), (64, 1000)]
+    parts, cu_q, cu_k, Qp, Kp, Vp = _packed(seqs, H, Hkv, d)
+    scale = 1.0 / np.sqrt(d)
+    Q, K, V = (P.to_dev(x, "bf16") for x in (Qp, Kp, Vp))
+    ws = mala.alloc_workspace(mala.varlen_workspace_bytes(cu_q, H, Hkv, d), "cuda")
+    O, LSE = mala.mala_fwd_varlen(Q, K, V, cu_q, cu_k, scale, tau, workspace=ws)
+    torch.cuda.synchronize()
+    assert mala.read_device_error(ws) == 0
+    st = mala.get_stats(ws)
+    O, LSE = O.float().cpu().numpy(), LSE.cpu().numpy()
+    legal = retained = 0
+    for s, (Qc, Ks, Vs, w) in enumerate(parts):
+        if Qc.shape[1] == 0:
+            continue
+        Qd, Kd, Vd = (P.to_dev(x, "bf16") for x in (Qc, Ks, Vs))
+        wss = mala.alloc_workspace(mala.fwd_workspace_bytes(1, H, Hkv, Qc.shape[1], d), "cuda")
+        Os, Ls = mala.mala_fwd_prefill(Qd, Kd, Vd, scale, tau, workspace=wss)
+        torch.cuda.synchronize()
+        sst = mala.get_stats(wss)
+        legal += sst["legal_tiles"]
+        retained += sst["retained_tiles"]
+        rows = slice(cu_q[s], cu_q[s + 1])
+        np.testing.assert_array_equal(O[rows], Os.float().cpu().numpy()[0])
+        np.testing.assert_array_equal(LSE[:, rows], Ls.cpu().numpy()[0])
+    assert st["legal_tiles"] == legal and st["retained_tiles"] == retained
+
+
+def test_varlen_parity_with_oracle(orc, mala):
+    H, Hkv, d = 2, 1, 64
+    seqs = [(200, 450), (90, 90), (333, 333)]
+    parts, cu_q, cu_k, Qp, Kp, Vp = _packed(seqs, H, Hkv, d)
+    scale = 1.0 / np.sqrt(d)
+    Q, K, V = (P.to_dev(x, "bf16") for x in (Qp, Kp, Vp))
+    O, LSE = mala.mala_fwd_varlen(Q, K, V, cu_q, cu_k, scale, 1.0)
+    torch.cuda.synchronize()
+    O, LSE = O.float().cpu().numpy(), LSE.cpu().numpy()
+    for s, (Qc, Ks, Vs, w) in enumerate(parts):
+        # the GPU's decisions for this sequence (from its own prefill call) are replayed
+        _, _, mask = run_prefill(mala, Qc, Ks, Vs, w, 1.0)
+        legal = prefill_legal(1, H, Qc.shape[1], Ks.shape[1])
+        force = np.where(legal, mask.astype(np.int16), -1).astype(np.int8)
+        oO, oLSE, _, _ = orc.mala_prefill(Qc, Ks, Vs, scale, 1.0, force=force)
+        rows = slice(cu_q[s], cu_q[s + 1])
+        P.check_output(O[rows][None], oO, np.ones(oO.shape[:-1], bool))
+        assert np.abs(LSE[:, rows] - oLSE[0]).max() < P.LSE_ABS

@@ -87,6 +87,13 @@ def test_invalid_arguments_are_rejected_before_any_launch(lib):
                       0.1, 1.0, 0, None, 0, None, None) == 1
     # statistics need a workspace and an output
     assert L.mala_get_stats(None, None, None) == 1
+    # packed batches: offsets must start at 0 and every sequence needs N_k >= N_q
+    ia = lambda xs: (ctypes.c_int * len(xs))(*xs)
+    args = (1, 4, 2, 128, 0, 0.1, 1.0, 0, vp(), 1 << 20, None)
+    assert L.mala_fwd_varlen(vp(), vp(), vp(), vp(), vp(), ia([5, 10]), ia([0, 10]), *args) == 1
+    assert L.mala_fwd_varlen(vp(), vp(), vp(), vp(), vp(), ia([0, 10]), ia([0, 5]), *args) == 1
+    assert L.mala_fwd_varlen_workspace_bytes(ia([0, 300, 300, 557]), 3, 4, 2, 128, 0) == \
+        256 + (3 + 0 + 3) * 32
     # workspace too small (checked before any CUDA call)
     assert L.mala_fwd(vp(), vp(), vp(), vp(), vp(), 1, 4, 2, 128, 128, 0, 0.1, 1.0, 0, vp(), 8,
                       None, None) == 5
