@@ -29,6 +29,9 @@ available; these synthetic distributions stand in for them):
                   28 * sum_h q_h / |q_h| + 0.1 N(0, 1) over the group's heads
 * ``sinkband128k`` B=1, H=8, H_kv=1, L=131072, d=128, bf16; sink + band states as
                   ``sinkband32k`` (one rank of an 8-way head-sharded 64/8-head model)
+* ``prevvar8k``   B=1, H=16, H_kv=4, L=8192, d=128, bf16; "previous-token" heads whose
+                  strength (8 + 12 u_h) and noise (0.3 + 0.7 v_h) vary per head and seed
+                  (the matched-work study's input)
 * ``prevtok32k``  B=1, H=32, H_kv=8, L=32768, d=128, bf16; concentrated "previous-token"
                   heads: q_t = 18 sqrt(d) K_{t-1} / |K_{t-1}|^2 + 0.3 N(0, 1), so the
                   previous token's scaled score is ~18 and the rest of the row is a flat
@@ -87,6 +90,8 @@ WORKLOADS = {
     # concentrated heads: each query copies the previous token's key (a "previous-token"
     # head), so most off-diagonal tiles fall below tau / L_q and are skipped
     "prevtok32k": Workload("prevtok32k", 1, 32, 8, 32768, 128, "bf16", "prev_token", 6),
+    # previous-token heads of varying concentration at 8K: the matched-work study input
+    "prevvar8k": Workload("prevvar8k", 1, 16, 4, 8192, 128, "bf16", "prev_token_var", 8),
 }
 
 
@@ -196,6 +201,22 @@ def make_training(w: Workload, L: int | None = None) -> dict:
         Q = np.empty((B, L, H, d), dtype=np.float32)
         for h in range(H):
             Q[:, :, h] = 0.5 * u[:, :, h // G] + math.sqrt(0.75) * n[:, :, h]
+        Q = _round(Q, w.dtype)
+    elif w.structure == "prev_token_var":
+        # previous-token heads of varying concentration: head h uses strength
+        # s0_h = 8 + 12 u_h and noise b_h = 0.3 + 0.7 v_h (u, v uniform, drawn from the
+        # seed), otherwise as "prev_token"; weak heads keep a heavier, less flat tail
+        rng = _rng(w.seed, _PLANT)
+        s0 = 8.0 + 12.0 * rng.random(H)
+        bn = 0.3 + 0.7 * rng.random(H)
+        n = normal(w.seed, _NOISE, (B, L, H, d), "fp32")
+        G = H // Hkv
+        kp = K[:, :-1].astype(np.float64)
+        kp = kp * (math.sqrt(d) / np.maximum((kp * kp).sum(-1, keepdims=True), 1e-6))
+        Q = np.empty((B, L, H, d), dtype=np.float32)
+        for h in range(H):
+            Q[:, :, h] = bn[h] * n[:, :, h]
+            Q[:, 1:, h] += (s0[h] * kp[:, :, h // G]).astype(np.float32)
         Q = _round(Q, w.dtype)
     elif w.structure == "prev_token":
         # q_t = s0 sqrt(d) K_{t-1} / |K_{t-1}|^2 + b n_t: the scaled score of the previous
