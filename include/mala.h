@@ -207,6 +207,17 @@ int mala_decode_num_splits(int B, int H, int H_kv, int Nk);
 mala_status mala_read_device_error(const void* workspace, void* stream, uint32_t* out,
                                    int clear);
 
+/*
+ * mala_selftest_wait_timeout - test hook for the failure handling of the kernels' waits
+ * (the page has no counterpart).  Launches one CTA whose single thread waits on an
+ * mbarrier that nothing ever arrives on, using the same bounded wait as the kernels
+ * (wall-clock budget budget_ns, 1 ns .. 10 s).  The wait runs out and records
+ * MALA_ERR_TIMEOUT (low byte; upper bits name the wait) in the workspace error word, which
+ * this call zeroes first; read it with mala_read_device_error().  No fault, trap or hang:
+ * the kernel returns and the context stays usable.
+ */
+mala_status mala_selftest_wait_timeout(void* workspace, uint64_t budget_ns, void* stream);
+
 /* Sets the wall-clock budget of every internal wait (default 2 s; test hook). */
 mala_status mala_set_wait_budget_ns(uint64_t ns);
 

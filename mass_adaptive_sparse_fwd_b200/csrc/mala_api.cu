@@ -13,6 +13,7 @@
 
 #include "mala.h"
 #include "mala_common.cuh"
+#include "sm100.cuh"
 
 namespace mala {
 cudaError_t launch_fwd_bf16(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
@@ -111,6 +112,24 @@ mala_status with_workspace(void* workspace, size_t ws_bytes, size_t need, cudaSt
   return st;
 }
 
+// Self-test of the bounded waits: one thread waits on an mbarrier that nothing arrives
+// on, so the wait runs out after `budget_ns` and records MALA_ERR_TIMEOUT in `err`.
+__global__ void selftest_wait_kernel(uint32_t* err, uint64_t budget_ns) {
+  __shared__ uint64_t bar;
+  __shared__ uint32_t flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const AbortState st{&flag, err, budget_ns, 0xF00u};
+    (void)mbar_wait(&bar, 0, st, 1);
+  }
+  __syncthreads();
+}
+
 }  // namespace mala
 
 using namespace mala;
@@ -149,6 +168,17 @@ mala_status mala_read_device_error(const void* workspace, void* stream, uint32_t
   if (clear && cudaMemsetAsync(const_cast<void*>(workspace), 0, 4, s) != cudaSuccess)
     return MALA_ERR_CUDA;
   return MALA_OK;
+}
+
+mala_status mala_selftest_wait_timeout(void* workspace, uint64_t budget_ns, void* stream) {
+  if (!workspace || budget_ns == 0 || budget_ns > 10000000000ull) return MALA_ERR_INVALID_ARG;
+  if (!aligned16(workspace)) return MALA_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint32_t* hdr = static_cast<uint32_t*>(workspace);
+  if (cudaMemsetAsync(hdr + kHdrError, 0, sizeof(uint32_t), s) != cudaSuccess)
+    return MALA_ERR_CUDA;
+  selftest_wait_kernel<<<1, 32, 0, s>>>(hdr + kHdrError, budget_ns);
+  return cudaGetLastError() == cudaSuccess ? MALA_OK : MALA_ERR_CUDA;
 }
 
 mala_status mala_get_stats(const void* workspace, void* stream, mala_stats* out) {

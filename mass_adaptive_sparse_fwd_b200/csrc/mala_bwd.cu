@@ -234,7 +234,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         AbortState drain = ast;
         uint32_t zero = 0;
         drain.flag = &zero;
-        drain.budget_ns = 200000000ull;
+        drain.budget_ns = kTeardownBudgetNs;
         if (nu > 0) mbar_wait(&sh.kv_full, (nu - 1) & 1, drain, 4);
         for (uint32_t cc = (c > NQ ? c - NQ : 0); cc < c; ++cc)
           mbar_wait(&sh.q_full[cc % NQ], (cc / NQ) & 1, drain, 4);
@@ -352,6 +352,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       AbortState fin = ast;
       uint32_t zero = 0;
       fin.flag = &zero;
+      fin.budget_ns = kTeardownBudgetNs;
       mbar_wait(&sh.final_bar, 0, fin, 18);
     }
   } else if (warp >= 4 && warp < 12) {

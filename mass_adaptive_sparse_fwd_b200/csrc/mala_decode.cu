@@ -195,7 +195,7 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, 1)
         AbortState drain = ast;
         uint32_t zero = 0;
         drain.flag = &zero;
-        drain.budget_ns = 200000000ull;
+        drain.budget_ns = kTeardownBudgetNs;
         for (uint32_t cc = (c > NK ? c - NK : 0); cc < c; ++cc)
           mbar_wait(&sh.k_full[cc % NK], (cc / NK) & 1, drain, 2);
       }
@@ -228,7 +228,7 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, 1)
         AbortState drain = ast;
         uint32_t zero = 0;
         drain.flag = &zero;
-        drain.budget_ns = 200000000ull;
+        drain.budget_ns = kTeardownBudgetNs;
         for (uint32_t cc = (c > NV ? c - NV : 0); cc < c; ++cc)
           mbar_wait(&sh.v_full[cc % NV], (cc / NV) & 1, drain, 5);
       }

@@ -217,7 +217,7 @@ __global__ void __launch_bounds__(384, 1)
         AbortState drain = ast;
         uint32_t zero = 0;
         drain.flag = &zero;
-        drain.budget_ns = 200000000ull;
+        drain.budget_ns = kTeardownBudgetNs;
         for (uint32_t cc = (c > NS ? c - NS : 0); cc < c; ++cc) {
           mbar_wait(&sh.k_full[cc % NS], (cc / NS) & 1, drain, 4);
           mbar_wait(&sh.v_full[cc % NS], (cc / NS) & 1, drain, 4);
@@ -312,6 +312,7 @@ __global__ void __launch_bounds__(384, 1)
       AbortState fin = ast;
       uint32_t zero = 0;
       fin.flag = &zero;
+      fin.budget_ns = kTeardownBudgetNs;
       mbar_wait(&sh.final_bar, 0, fin, 17);
     }
   } else if (warp >= 4) {

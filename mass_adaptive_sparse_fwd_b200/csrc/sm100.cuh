@@ -35,6 +35,11 @@ struct AbortState {
   uint32_t site_base;       // identifies the kernel in the recorded error
 };
 
+// Budget of the teardown waits (in-flight loads drained, own MMAs completed before TMEM
+// is freed): fixed and generous, independent of the per-wait budget, so that a short test
+// budget can never free resources that the hardware is still using.
+constexpr uint64_t kTeardownBudgetNs = 200000000ull;
+
 __device__ __forceinline__ void record_timeout(const AbortState& st, uint32_t site) {
   *st.flag = 1u;
   if (st.err) {

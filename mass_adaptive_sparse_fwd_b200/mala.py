@@ -26,6 +26,7 @@ TILE = 128
 
 EXPORTED = ("mala_fwd", "mala_fwd_prefill", "mala_fwd_varlen", "mala_bwd", "mala_decode",
             "mala_decode_noalloc", "mala_get_stats", "mala_fwd_varlen_workspace_bytes",
+            "mala_selftest_wait_timeout",
             "mala_fwd_workspace_bytes",
             "mala_bwd_workspace_bytes", "mala_decode_workspace_bytes", "mala_decode_num_splits",
             "mala_read_device_error", "mala_set_wait_budget_ns", "mala_status_string",
@@ -79,6 +80,8 @@ def load_library(path: str = _LIB_PATH) -> ctypes.CDLL:
     lib.mala_decode_num_splits.restype = ci
     lib.mala_read_device_error.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_uint32), ci]
     lib.mala_set_wait_budget_ns.argtypes = [ctypes.c_uint64]
+    lib.mala_selftest_wait_timeout.argtypes = [vp, ctypes.c_uint64, vp]
+    lib.mala_selftest_wait_timeout.restype = ci
     lib.mala_get_stats.argtypes = [vp, vp, ctypes.POINTER(MalaStats)]
     lib.mala_get_stats.restype = ci
     lib.mala_status_string.argtypes = [ci]
@@ -275,6 +278,12 @@ def get_stats(workspace: torch.Tensor, stream=None) -> dict:
                                                  ctypes.byref(out)))
     return {"legal_tiles": out.legal_tiles, "retained_tiles": out.retained_tiles,
             "v_tiles_loaded": out.v_tiles_loaded}
+
+
+def selftest_wait_timeout(workspace: torch.Tensor, budget_ns: int, stream=None):
+    """Runs the bounded-wait self-test kernel (a wait that nothing satisfies)."""
+    _check("mala_selftest_wait_timeout",
+           _lib.mala_selftest_wait_timeout(_ptr(workspace), int(budget_ns), _stream(stream)))
 
 
 def set_wait_budget_ns(ns: int):
