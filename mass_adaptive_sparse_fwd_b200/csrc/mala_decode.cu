@@ -139,6 +139,25 @@ __device__ __forceinline__ void unit_coords(const DecParams& p, int u, int& b, i
   t_hi = static_cast<int>(static_cast<long long>(s + 1) * p.T / p.S);
 }
 
+// Applies the previous tile's decision of head dh to the normaliser once that tile's
+// per-warp row sums are published: l = l alpha + sum_w rowsum_w beta_w (lane (dw, dh) holds
+// segment dw's beta; the 8 segment lanes of a head reduce by shuffles).  Warp-collective.
+template <int CW>
+__device__ __forceinline__ void close_prev(const float (&rsum)[8][4], int dw, int dh,
+                                           float mnew_prev, float alpha_prev, float beta_prev,
+                                           bool& k_prev, float& m_h, float& l_h) {
+  const float sv = (dw < CW) ? rsum[dw][dh] : 0.f;
+  float sum = k_prev ? sv * beta_prev : 0.f;
+  sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+  sum += __shfl_xor_sync(0xffffffffu, sum, 2);
+  sum += __shfl_xor_sync(0xffffffffu, sum, 4);
+  if (k_prev) {
+    l_h = l_h * alpha_prev + sum;
+    m_h = mnew_prev;
+  }
+  k_prev = false;
+}
+
 template <int D, bool kScreen>
 __global__ void __launch_bounds__(DecCfg<D>::THREADS, 1)
     mala_decode_kernel(const __grid_constant__ CUtensorMap tmK,
@@ -271,6 +290,10 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, 1)
         qb[ks][1] = *reinterpret_cast<const uint32_t*>(&sh.qs[hh][c0 + 8]);
       }
       float m_h = NEG_INF, l_h = 0.f;  // running state of head dh (online, log2 units)
+      // the previous tile's decision for head dh, applied to l once its row sums arrive
+      bool k_prev = false;
+      float mnew_prev = NEG_INF, alpha_prev = 1.f, beta_prev = 0.f;
+      float ps_prev[2] = {0.f, 0.f};  // this warp's row sums of the previous tile
       // O^T accumulators: warp owns head-dim rows [16 MB w, 16 MB (w+1))
       float acc[MB][4];
 #pragma unroll
@@ -283,7 +306,6 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, 1)
           const int t = t_hi - 1 - n;
           const uint32_t slot = (n_glob + n) % kPR;
           const int kst = kc % NK;
-          const float cut = m_h + __log2f(l_h) + p.thr2;
           // A failed wait only raises the abort flag; the consumers leave the loop
           // together, right after their next named barrier.
           const bool got = mbar_wait_warp(&sh.k_full[kst], (kc / NK) & 1, ast, 10);
@@ -308,9 +330,8 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, 1)
           __syncwarp();
           if (lane == 0) mbar_arrive(&sh.k_empty[kst]);
           ++kc;
-          // log2-domain scores (keys past the end masked), this warp's maxima and
-          // P relative to them, written before the decision: thread columns are heads
-          // h0 and h0 + 1, rows are keys
+          // log2-domain scores (keys past the end masked) and this warp's maxima: thread
+          // columns are heads h0 and h0 + 1, rows are keys
           const int h0 = (lane & 3) * 2;
           float mx[2] = {NEG_INF, NEG_INF};
 #pragma unroll
@@ -328,71 +349,46 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, 1)
             mx[0] = fmaxf(mx[0], __shfl_xor_sync(0xffffffffu, mx[0], o));
             mx[1] = fmaxf(mx[1], __shfl_xor_sync(0xffffffffu, mx[1], o));
           }
-          float ps[2] = {0.f, 0.f};
-#pragma unroll
-          for (int kb = 0; kb < KB; ++kb)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int c = e & 1, hh = h0 + c;
-              const float mu = (mx[c] == NEG_INF) ? 0.f : mx[c];
-              const float pv = fast_exp2(sc[kb][e] - mu);
-              ps[c] += pv;
-              if (hh < G)
-                sh.P[slot][hh][warp * (16 * KB) + kb * 16 + (lane >> 2) + (e >> 1) * 8] = pv;
-            }
-#pragma unroll
-          for (int o = 4; o < 32; o <<= 1) {
-            ps[0] += __shfl_xor_sync(0xffffffffu, ps[0], o);
-            ps[1] += __shfl_xor_sync(0xffffffffu, ps[1], o);
-          }
+          // the tile's only barrier publishes this tile's per-warp maxima together with
+          // the previous tile's per-warp row sums; it also orders the P, beta and alpha of
+          // older tiles before their P.V below
           const int rb = n & 1;
           if (lane < 2) {  // lanes 0, 1 hold heads 0-1 and 2-3
             sh.rmax[rb][warp][lane * 2] = mx[0];
             sh.rmax[rb][warp][lane * 2 + 1] = mx[1];
-            sh.rsum[rb][warp][lane * 2] = ps[0];
-            sh.rsum[rb][warp][lane * 2 + 1] = ps[1];
+            sh.rsum[rb][warp][lane * 2] = ps_prev[0];
+            sh.rsum[rb][warp][lane * 2 + 1] = ps_prev[1];
           }
-          // the tile's only barrier; it also orders the P, beta and alpha of older
-          // tiles before their P.V below
           named_bar_sync(1, NT);
           if (*ast.flag) { ok = false; break; }
-          // retention test of head dh (Eq. 3 with L_0 = N_k) on the tile maximum, and
-          // the normaliser update l = l alpha + sum_w rowsum_w 2^(max_w - m_new)
+          close_prev<CW>(sh.rsum[rb], dw, dh, mnew_prev, alpha_prev, beta_prev, k_prev, m_h, l_h);
+          // retention test of head dh (Eq. 3 with L_0 = N_k) on the tile maximum
           const float mv = (dw < CW) ? sh.rmax[rb][dw][dh] : NEG_INF;
-          const float sv = (dw < CW) ? sh.rsum[rb][dw][dh] : 0.f;
           float tmax = mv;
           tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 1));
           tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 2));
           tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 4));
           bool k = dh < G;
-          if (kScreen && k) k = (l_h == 0.f) || (tmax >= cut);
+          if (kScreen && k) k = (l_h == 0.f) || (tmax >= m_h + __log2f(l_h) + p.thr2);
           const uint32_t bal = __ballot_sync(0xffffffffu, k);
           const uint32_t keep = (bal & 1u) | ((bal >> 7) & 2u) | ((bal >> 14) & 4u) |
                                 ((bal >> 21) & 8u);
-          if (bal) {  // warp-uniform: some head keeps the tile
-            float mnew = m_h, alpha = 1.f, beta = 0.f;
-            if (k) {
-              if (tmax > m_h + 8.0f) {
-                mnew = tmax;
-                alpha = fast_exp2(m_h - tmax);  // 0 on the first retained tile
-              }
-              beta = fast_exp2(mv - mnew);      // 0 for a segment with no valid key
+          k_prev = k;
+          if (k) {  // the normaliser update itself waits for the row sums (next barrier)
+            mnew_prev = m_h;
+            alpha_prev = 1.f;
+            if (tmax > m_h + 8.0f) {
+              mnew_prev = tmax;
+              alpha_prev = fast_exp2(m_h - tmax);  // 0 on the first retained tile
             }
-            float sum = sv * beta;
-            sum += __shfl_xor_sync(0xffffffffu, sum, 1);
-            sum += __shfl_xor_sync(0xffffffffu, sum, 2);
-            sum += __shfl_xor_sync(0xffffffffu, sum, 4);
-            if (k) {
-              l_h = l_h * alpha + sum;
-              m_h = mnew;
-            }
-            if (warp == 0) {
-              if (dw < CW) sh.beta[slot][dw][dh] = beta;
-              if (dw == 0) sh.alpha[slot][dh] = alpha;
-            }
+            beta_prev = fast_exp2(mv - mnew_prev);  // 0 for a segment with no valid key
           }
-          if (warp == 0 && p.tile_mask && dw == 0 && dh < G)
-            p.tile_mask[(static_cast<size_t>(b) * p.H + g * G + dh) * p.T + t] = k ? 1 : 0;
+          if (warp == 0) {
+            if (dw < CW) sh.beta[slot][dw][dh] = k ? beta_prev : 0.f;
+            if (dw == 0) sh.alpha[slot][dh] = k ? alpha_prev : 1.f;
+            if (p.tile_mask && dw == 0 && dh < G)
+              p.tile_mask[(static_cast<size_t>(b) * p.H + g * G + dh) * p.T + t] = k ? 1 : 0;
+          }
           // hand the decision to the V producer (ring slot must be free)
           if (tid == 0) {
             st_legal += static_cast<uint32_t>(G);
@@ -403,10 +399,39 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, 1)
             sh.keep[slot] = keep;
             if (free_slot) mbar_arrive(&sh.dec_full[slot]);
           }
+          // P of a kept tile, relative to this warp's own maxima (a head that skips the
+          // tile gets beta = 0), and this warp's row sums for the next barrier
+          ps_prev[0] = 0.f;
+          ps_prev[1] = 0.f;
+          if (bal) {
+#pragma unroll
+            for (int kb = 0; kb < KB; ++kb)
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const int c = e & 1, hh = h0 + c;
+                const float mu = (mx[c] == NEG_INF) ? 0.f : mx[c];
+                const float pv = fast_exp2(sc[kb][e] - mu);
+                ps_prev[c] += pv;
+                if (hh < G)
+                  sh.P[slot][hh][warp * (16 * KB) + kb * 16 + (lane >> 2) + (e >> 1) * 8] = pv;
+              }
+#pragma unroll
+            for (int o = 4; o < 32; o <<= 1) {
+              ps_prev[0] += __shfl_xor_sync(0xffffffffu, ps_prev[0], o);
+              ps_prev[1] += __shfl_xor_sync(0xffffffffu, ps_prev[1], o);
+            }
+          }
         } else if (n == nt) {
-          // orders the last tile's P, beta, alpha and keep before the P.V that follow
+          // publish the last tile's row sums and close it; this barrier also orders its P,
+          // beta, alpha and keep before the P.V that follow
+          const int rb = n & 1;
+          if (lane < 2) {
+            sh.rsum[rb][warp][lane * 2] = ps_prev[0];
+            sh.rsum[rb][warp][lane * 2 + 1] = ps_prev[1];
+          }
           named_bar_sync(1, NT);
           if (*ast.flag) { ok = false; break; }
+          close_prev<CW>(sh.rsum[rb], dw, dh, mnew_prev, alpha_prev, beta_prev, k_prev, m_h, l_h);
         }
         // P.V of the tile decided kLag iterations ago
         if (n >= kLag) {
