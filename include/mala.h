@@ -223,7 +223,7 @@ mala_status mala_set_wait_budget_ns(uint64_t ns);
 
 const char* mala_status_string(mala_status s);
 
-/* Library version, e.g. 100 = 0.1.0. */
+/* Library version: 200 = 0.2.0 (adds mala_fwd_prefill, mala_fwd_varlen, mala_get_stats). */
 int mala_version(void);
 
 #ifdef __cplusplus

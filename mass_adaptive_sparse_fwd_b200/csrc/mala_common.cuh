@@ -16,7 +16,6 @@ enum HeaderWord : int {
   kHdrSched0 = 1,     // persistent-scheduler counters
   kHdrSched1 = 2,
   kHdrSched2 = 3,
-  kHdrTickets = 16,   // decode merge tickets start here (not used by fwd/bwd)
 };
 
 // Call statistics in the workspace header: three uint64 counters at this byte offset,

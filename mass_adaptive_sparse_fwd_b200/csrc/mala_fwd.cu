@@ -177,8 +177,6 @@ __global__ void __launch_bounds__(384, 1)
       tma_prefetch_desc(&tmV);
       uint32_t c = 0;                  // K/V tiles issued (all units)
       uint32_t nq[2] = {0, 0};         // Q loads issued per slot
-      int last_q_stage_used = 0;
-      (void)last_q_stage_used;
       bool ok = true;
       for (uint32_t k = 0; ok; ++k) {
         const int ring = k & 1;
