@@ -428,6 +428,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           const float4* c4 = reinterpret_cast<const float4*>(sh.cut2[wg]);
           float ymax = NEG_INF;
           if (qlo < 0) {
+            // four independent three-input max chains
+            float y4[4] = {NEG_INF, NEG_INF, NEG_INF, NEG_INF};
 #pragma unroll
             for (int a = 0; a < 2; ++a)
 #pragma unroll
@@ -438,9 +440,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 const float y1 = fmaf(__uint_as_float(sv[1]), p.scale_log2, -cv.y);
                 const float y2 = fmaf(__uint_as_float(sv[2]), p.scale_log2, -cv.z);
                 const float y3 = fmaf(__uint_as_float(sv[3]), p.scale_log2, -cv.w);
-                ymax = fmax3(ymax, y0, y1);
-                ymax = fmax3(ymax, y2, y3);
+                y4[(e4 & 1) * 2] = fmax3(y4[(e4 & 1) * 2], y0, y1);
+                y4[(e4 & 1) * 2 + 1] = fmax3(y4[(e4 & 1) * 2 + 1], y2, y3);
               }
+            ymax = fmaxf(fmaxf(y4[0], y4[1]), fmaxf(y4[2], y4[3]));
           } else {
 #pragma unroll
             for (int a = 0; a < 2; ++a)

@@ -83,6 +83,11 @@ struct Unit {
   int L, off;        // the sequence's query rows and causal offset
 };
 
+// Whether slot s of the unit holds a head (constant-index access keeps Unit in registers).
+__device__ __forceinline__ bool slot_active(const Unit& w, int s) {
+  return s == 0 ? w.active[0] : w.active[1];
+}
+
 // Last key block holding a legal key of the unit's query block (its last row's position).
 __device__ __forceinline__ int last_key_tile(const Unit& w) {
   const int q_last = min(w.i * kTile + kTile - 1, w.L - 1);
@@ -187,7 +192,7 @@ __global__ void __launch_bounds__(384, 1)
         if (u >= p.n_units) break;
         const Unit w = decode_unit(p, u);
         for (int s = 0; s < 2 && ok; ++s) {
-          if (!w.active[s]) continue;
+          if (!slot_active(w, s)) continue;
           if (nq[s] > 0 && !(ok = mbar_wait(&sh.q_empty[s], (nq[s] - 1) & 1, ast, 2))) break;
           mbar_arrive_expect_tx(&sh.q_full[s], C::TILE_BYTES);
           for (int x = 0; x < C::BOXES; ++x)
@@ -252,7 +257,7 @@ __global__ void __launch_bounds__(384, 1)
         if (u >= p.n_units) break;
         const Unit w = decode_unit(p, u);
         for (int s = 0; s < 2 && ok; ++s) {
-          if (!w.active[s]) continue;
+          if (!slot_active(w, s)) continue;
           ok = mbar_wait(&sh.q_full[s], nq[s] & 1, ast, 11);
           ++nq[s];
         }
@@ -265,13 +270,13 @@ __global__ void __launch_bounds__(384, 1)
           if (!(ok = mbar_wait(&sh.k_full[st], (c / NS) & 1, ast, 12))) break;
           tc_fence_after();
           for (int s = 0; s < 2; ++s)
-            if (w.active[s]) issue_qk(s, st);
+            if (slot_active(w, s)) issue_qk(s, st);
         }
         for (int t = 0; t < n && ok; ++t, ++c) {
           const int st = c % NS;
           bool v_ready = false, k_next_ready = false;
           for (int s = 0; s < 2 && ok; ++s) {
-            if (!w.active[s]) continue;
+            if (!slot_active(w, s)) continue;
             if (!(ok = mbar_wait(&sh.p_full[s], np[s] & 1, ast, 13))) break;
             ++np[s];
             tc_fence_after();
@@ -303,7 +308,7 @@ __global__ void __launch_bounds__(384, 1)
         }
         if (!ok) break;
         for (int s = 0; s < 2; ++s)
-          if (w.active[s]) umma_commit(&sh.q_empty[s]);
+          if (slot_active(w, s)) umma_commit(&sh.q_empty[s]);
       }
       // wait for every MMA this thread issued before TMEM is released
       umma_commit(&sh.final_bar);
@@ -334,7 +339,7 @@ __global__ void __launch_bounds__(384, 1)
       mbar_arrive(&sh.sched_empty[ring]);
       if (u >= p.n_units) break;
       const Unit w = decode_unit(p, u);
-      if (!w.active[s]) continue;
+      if (!slot_active(w, s)) continue;
       const int h = w.h0 + s;
       const int q = w.i * kTile + r;
       const bool valid = q < w.L;
@@ -378,10 +383,19 @@ __global__ void __launch_bounds__(384, 1)
                   rraw = fmaxf(rraw, col <= lim ? __uint_as_float(v[a][e]) : NEG_INF);
                 }
             } else {
+              // four independent three-input max chains (a single chain would serialise
+              // 64 dependent max operations per 64 columns)
+              float r0 = rraw, r1 = NEG_INF, r2 = NEG_INF, r3 = NEG_INF;
 #pragma unroll
               for (int a = 0; a < 2; ++a)
 #pragma unroll
-                for (int e = 0; e < 32; ++e) rraw = fmaxf(rraw, __uint_as_float(v[a][e]));
+                for (int e = 0; e < 32; e += 8) {
+                  r0 = fmax3(r0, __uint_as_float(v[a][e]), __uint_as_float(v[a][e + 1]));
+                  r1 = fmax3(r1, __uint_as_float(v[a][e + 2]), __uint_as_float(v[a][e + 3]));
+                  r2 = fmax3(r2, __uint_as_float(v[a][e + 4]), __uint_as_float(v[a][e + 5]));
+                  r3 = fmax3(r3, __uint_as_float(v[a][e + 6]), __uint_as_float(v[a][e + 7]));
+                }
+              rraw = fmaxf(fmaxf(r0, r1), fmaxf(r2, r3));
             }
           }
         }
@@ -426,7 +440,7 @@ __global__ void __launch_bounds__(384, 1)
         // pass 2: P = exp2(s * scale * log2(e) - m), 32 keys at a time, packed into the
         // first 64 columns of the same TMEM region (each store lands on columns this
         // thread has already read)
-        float psum = 0.f;
+        float ps0 = 0.f, ps1 = 0.f;  // two independent partial sums
 #pragma unroll
         for (int cc = 0; cc < 4; ++cc) {
           uint32_t v[32];
@@ -444,12 +458,13 @@ __global__ void __launch_bounds__(384, 1)
           for (int e = 0; e < 16; ++e) {
             const float p0 = fast_exp2(fmaf(__uint_as_float(v[2 * e]), p.scale_log2, -m_use));
             const float p1 = fast_exp2(fmaf(__uint_as_float(v[2 * e + 1]), p.scale_log2, -m_use));
-            psum += p0 + p1;
+            if (e & 1) ps1 += p0 + p1; else ps0 += p0 + p1;
             pk[e] = pack_bf16(p0, p1);
           }
           tmem_st16(tS + cc * 16, pk);
         }
         tmem_wait_st();
+        const float psum = ps0 + ps1;
         l = l * alpha + psum;
         m2 = m_new;
         if (r == 0) sh.dec[s] = 1;
