@@ -282,12 +282,24 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           if (!(ok = mbar_wait(&sh.p_full, ntile & 1, ast, 13))) break;
           tc_fence_after();
           const bool keep = sh.dec != 0;
-          // a skipped tile's Q stage was read only by its S^T MMA, which has completed:
-          // release it now so that the producer's next Q load starts a step earlier
-          if (!keep) umma_commit(&sh.q_empty[st]);
-          // dO(c) is loaded for every tile; its stage is released after dP^T / dV
-          if (!(ok = mbar_wait(&sh.do_full, c & 1, ast, 20))) break;
-          if (keep) {
+          if (!keep) {
+            // Skipped tile: its Q stage was read only by its own S^T MMA, which completed
+            // before the decision, and its dO by no MMA, so both stages go back at once
+            // with plain arrivals (no tensor-core work of this tile is pending on them);
+            // dO is released before the next S^T issue so the single-stage dO ring's next
+            // load starts as early as possible.
+            mbar_arrive(&sh.q_empty[st]);
+            // the dO load of this tile must have landed before its stage is handed back
+            if (!(ok = mbar_wait(&sh.do_full, c & 1, ast, 20))) break;
+            mbar_arrive(&sh.do_empty);
+            if (n + 1 < w.ntiles) {
+              const uint32_t c1 = c + 1;
+              if (!(ok = mbar_wait(&sh.q_full[c1 % NQ], (c1 / NQ) & 1, ast, 16))) break;
+              tc_fence_after();
+              issue_s(c1);
+            }
+          } else {
+            if (!(ok = mbar_wait(&sh.do_full, c & 1, ast, 20))) break;
             // dP^T reuses the columns of the previous dQ tile: wait for its drain
             if (ntile > 0 && !(ok = mbar_wait(&sh.dq_empty, (ntile - 1) & 1, ast, 14))) break;
             // first accumulation of the unit overwrites dK / dV: previous epilogue done
@@ -306,14 +318,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             for (int kk = 0; kk < 8; ++kk)
               umma_ts(tdV, tS + kk * 8, sdesc_sw128(adO + kk * 2048, 16384, 1024), id_acc,
                       (acc_started || kk > 0) ? 1u : 0u);
-          }
-          umma_commit(&sh.do_empty);
-          // next tile's S^T (after dV has consumed P^T from the same columns)
-          if (n + 1 < w.ntiles) {
-            const uint32_t c1 = c + 1;
-            if (!(ok = mbar_wait(&sh.q_full[c1 % NQ], (c1 / NQ) & 1, ast, 16))) break;
-            tc_fence_after();
-            issue_s(c1);
+            umma_commit(&sh.do_empty);  // after dP^T and dV have read dO
+            // next tile's S^T (after dV has consumed P^T from the same columns)
+            if (n + 1 < w.ntiles) {
+              const uint32_t c1 = c + 1;
+              if (!(ok = mbar_wait(&sh.q_full[c1 % NQ], (c1 / NQ) & 1, ast, 16))) break;
+              tc_fence_after();
+              issue_s(c1);
+            }
           }
           if (keep) {
             if (!(ok = mbar_wait(&sh.ds_full, nret & 1, ast, 17))) break;
