@@ -143,6 +143,8 @@ mala_status mala_bwd(const void* Q, const void* K, const void* V, const void* O,
  *   position N_k - 1); O [B,H,d] out; LSE [B,H] float32 out.
  *   Key tiles of 128; split s of S owns tiles [s*T/S, (s+1)*T/S) (integer division)
  *   and visits them newest first.  num_splits = 0 picks mala_decode_num_splits().
+ *   The bf16 path takes groups of up to 8 query heads per KV head (H / H_kv <= 8, else
+ *   MALA_ERR_UNSUPPORTED); the fp32 path takes any group.
  *   The retained support depends on the split count (the page says so).
  */
 mala_status mala_decode(const void* q, const void* Kc, const void* Vc, void* O, float* LSE,

@@ -85,12 +85,12 @@ struct DecShared {
   // P_t in fp32, rows = heads (>= G zero), each warp's keys relative to that warp's own
   // maximum; rows padded by 8 keys (bank spread of the P.V fragment loads)
   alignas(16) float P[kPR][8][kTile + 8];
-  float beta[kPR][8][4];              // [key segment][head]: 2^(segment max - new max)
-  float alpha[kPR][4];                // rescale of O at tile t, per head
+  float beta[kPR][8][8];              // [key segment][head]: 2^(segment max - new max)
+  float alpha[kPR][8];                // rescale of O at tile t, per head
   uint32_t keep[kPR];                 // bit h: head h retained tile t
-  // per-warp tile maxima and row sums (heads 0..3), double-buffered by tile parity
-  float rmax[2][8][4];
-  float rsum[2][8][4];
+  // per-warp tile maxima and row sums, [warp][head], double-buffered by tile parity
+  float rmax[2][8][8];
+  float rsum[2][8][8];
   uint32_t last_flag;
   uint32_t abort_flag;
 };
@@ -139,14 +139,14 @@ __device__ __forceinline__ void unit_coords(const DecParams& p, int u, int& b, i
   t_hi = static_cast<int>(static_cast<long long>(s + 1) * p.T / p.S);
 }
 
-// Applies the previous tile's decision of head dh to the normaliser once that tile's
-// per-warp row sums are published: l = l alpha + sum_w rowsum_w beta_w (lane (dw, dh) holds
+// Applies the previous tile's decision of head hd to the normaliser once that tile's
+// per-warp row sums are published: l = l alpha + sum_w rowsum_w beta_w (lane (dw, hd) holds
 // segment dw's beta; the 8 segment lanes of a head reduce by shuffles).  Warp-collective.
 template <int CW>
-__device__ __forceinline__ void close_prev(const float (&rsum)[8][4], int dw, int dh,
+__device__ __forceinline__ void close_prev(const float (&rsum)[8][8], int dw, int hd,
                                            float mnew_prev, float alpha_prev, float beta_prev,
                                            bool& k_prev, float& m_h, float& l_h) {
-  const float sv = (dw < CW) ? rsum[dw][dh] : 0.f;
+  const float sv = (dw < CW) ? rsum[dw][hd] : 0.f;
   float sum = k_prev ? sv * beta_prev : 0.f;
   sum += __shfl_xor_sync(0xffffffffu, sum, 1);
   sum += __shfl_xor_sync(0xffffffffu, sum, 2);
@@ -158,7 +158,8 @@ __device__ __forceinline__ void close_prev(const float (&rsum)[8][4], int dw, in
   k_prev = false;
 }
 
-template <int D, bool kScreen>
+// HS = head slots per decision lane: 1 for groups of up to 4 query heads, 2 for up to 8.
+template <int D, bool kScreen, int HS>
 __global__ void __launch_bounds__(DecCfg<D>::THREADS, 1)
     mala_decode_kernel(const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const DecParams p) {
@@ -266,9 +267,14 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, 1)
       const int row = (i / (kTile + 8)) % 8;
       if (row >= G) (&sh.P[0][0][0])[i] = 0.f;
     }
+    // scale factors of heads without a decision (padding, or heads 4..7 of a group of at
+    // most 4, whose slots are never written) stay finite: beta 0, alpha 1
+    for (int i = tid; i < kPR * 8 * 8; i += NT) (&sh.beta[0][0][0])[i] = 0.f;
+    for (int i = tid; i < kPR * 8; i += NT) (&sh.alpha[0][0])[i] = 1.f;
     // decision lanes: lane L of every consumer warp handles key segment (warp) dw and
-    // head dh; the per-head state m, l lives in the lanes of that head (replicated over
-    // the 8 segment lanes, and over warps: every warp takes the same decisions)
+    // heads dh and dh + 4 (a group has up to 8 heads); the per-head state m, l lives in
+    // the lanes of that head (replicated over the 8 segment lanes, and over warps: every
+    // warp takes the same decisions)
     const int dw = lane & 7, dh = lane >> 3;
     for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
       int b, g, s, t_lo, t_hi;
@@ -289,10 +295,12 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, 1)
         qb[ks][0] = *reinterpret_cast<const uint32_t*>(&sh.qs[hh][c0]);
         qb[ks][1] = *reinterpret_cast<const uint32_t*>(&sh.qs[hh][c0 + 8]);
       }
-      float m_h = NEG_INF, l_h = 0.f;  // running state of head dh (online, log2 units)
-      // the previous tile's decision for head dh, applied to l once its row sums arrive
-      bool k_prev = false;
-      float mnew_prev = NEG_INF, alpha_prev = 1.f, beta_prev = 0.f;
+      // running state (online, log2 units) of heads dh and dh + 4 (slots 0 and 1), and
+      // the previous tile's decision for them, applied to l once its row sums arrive
+      float m_h[2] = {NEG_INF, NEG_INF}, l_h[2] = {0.f, 0.f};  // slots [0, HS) used
+      bool k_prev[2] = {false, false};
+      float mnew_prev[2] = {NEG_INF, NEG_INF}, alpha_prev[2] = {1.f, 1.f};
+      float beta_prev[2] = {0.f, 0.f};
       float ps_prev[2] = {0.f, 0.f};  // this warp's row sums of the previous tile
       // O^T accumulators: warp owns head-dim rows [16 MB w, 16 MB (w+1))
       float acc[MB][4];
@@ -353,7 +361,7 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, 1)
           // the previous tile's per-warp row sums; it also orders the P, beta and alpha of
           // older tiles before their P.V below
           const int rb = n & 1;
-          if (lane < 2) {  // lanes 0, 1 hold heads 0-1 and 2-3
+          if (lane < 2 * HS) {  // lane c holds heads 2c and 2c + 1
             sh.rmax[rb][warp][lane * 2] = mx[0];
             sh.rmax[rb][warp][lane * 2 + 1] = mx[1];
             sh.rsum[rb][warp][lane * 2] = ps_prev[0];
@@ -361,34 +369,44 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, 1)
           }
           named_bar_sync(1, NT);
           if (*ast.flag) { ok = false; break; }
-          close_prev<CW>(sh.rsum[rb], dw, dh, mnew_prev, alpha_prev, beta_prev, k_prev, m_h, l_h);
-          // retention test of head dh (Eq. 3 with L_0 = N_k) on the tile maximum
-          const float mv = (dw < CW) ? sh.rmax[rb][dw][dh] : NEG_INF;
-          float tmax = mv;
-          tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 1));
-          tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 2));
-          tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 4));
-          bool k = dh < G;
-          if (kScreen && k) k = (l_h == 0.f) || (tmax >= m_h + __log2f(l_h) + p.thr2);
-          const uint32_t bal = __ballot_sync(0xffffffffu, k);
-          const uint32_t keep = (bal & 1u) | ((bal >> 7) & 2u) | ((bal >> 14) & 4u) |
-                                ((bal >> 21) & 8u);
-          k_prev = k;
-          if (k) {  // the normaliser update itself waits for the row sums (next barrier)
-            mnew_prev = m_h;
-            alpha_prev = 1.f;
-            if (tmax > m_h + 8.0f) {
-              mnew_prev = tmax;
-              alpha_prev = fast_exp2(m_h - tmax);  // 0 on the first retained tile
+          #pragma unroll
+          for (int hs = 0; hs < HS; ++hs)
+            close_prev<CW>(sh.rsum[rb], dw, dh + 4 * hs, mnew_prev[hs], alpha_prev[hs],
+                           beta_prev[hs], k_prev[hs], m_h[hs], l_h[hs]);
+          // retention test (Eq. 3 with L_0 = N_k) of heads dh and dh + 4 on the tile maxima
+          uint32_t keep = 0;
+#pragma unroll
+          for (int hs = 0; hs < HS; ++hs) {
+            const int hd = dh + 4 * hs;
+            const float mv = (dw < CW) ? sh.rmax[rb][dw][hd] : NEG_INF;
+            float tmax = mv;
+            tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 1));
+            tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 2));
+            tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 4));
+            bool k = hd < G;
+            if (kScreen && k)
+              k = (l_h[hs] == 0.f) || (tmax >= m_h[hs] + __log2f(l_h[hs]) + p.thr2);
+            const uint32_t bal = __ballot_sync(0xffffffffu, k);
+            keep |= ((bal & 1u) | ((bal >> 7) & 2u) | ((bal >> 14) & 4u) | ((bal >> 21) & 8u))
+                    << (4 * hs);
+            k_prev[hs] = k;
+            if (k) {  // the normaliser update itself waits for the row sums (next barrier)
+              mnew_prev[hs] = m_h[hs];
+              alpha_prev[hs] = 1.f;
+              if (tmax > m_h[hs] + 8.0f) {
+                mnew_prev[hs] = tmax;
+                alpha_prev[hs] = fast_exp2(m_h[hs] - tmax);  // 0 on the first retained tile
+              }
+              beta_prev[hs] = fast_exp2(mv - mnew_prev[hs]);  // 0 for a segment with no key
             }
-            beta_prev = fast_exp2(mv - mnew_prev);  // 0 for a segment with no valid key
+            if (warp == 0) {
+              if (dw < CW) sh.beta[slot][dw][hd] = k ? beta_prev[hs] : 0.f;
+              if (dw == 0) sh.alpha[slot][hd] = k ? alpha_prev[hs] : 1.f;
+              if (p.tile_mask && dw == 0 && hd < G)
+                p.tile_mask[(static_cast<size_t>(b) * p.H + g * G + hd) * p.T + t] = k ? 1 : 0;
+            }
           }
-          if (warp == 0) {
-            if (dw < CW) sh.beta[slot][dw][dh] = k ? beta_prev : 0.f;
-            if (dw == 0) sh.alpha[slot][dh] = k ? alpha_prev : 1.f;
-            if (p.tile_mask && dw == 0 && dh < G)
-              p.tile_mask[(static_cast<size_t>(b) * p.H + g * G + dh) * p.T + t] = k ? 1 : 0;
-          }
+          const uint32_t bal = keep;  // nonzero: some head keeps the tile (warp-uniform)
           // hand the decision to the V producer (ring slot must be free)
           if (tid == 0) {
             st_legal += static_cast<uint32_t>(G);
@@ -425,13 +443,16 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, 1)
           // publish the last tile's row sums and close it; this barrier also orders its P,
           // beta, alpha and keep before the P.V that follow
           const int rb = n & 1;
-          if (lane < 2) {
+          if (lane < 2 * HS) {
             sh.rsum[rb][warp][lane * 2] = ps_prev[0];
             sh.rsum[rb][warp][lane * 2 + 1] = ps_prev[1];
           }
           named_bar_sync(1, NT);
           if (*ast.flag) { ok = false; break; }
-          close_prev<CW>(sh.rsum[rb], dw, dh, mnew_prev, alpha_prev, beta_prev, k_prev, m_h, l_h);
+          #pragma unroll
+          for (int hs = 0; hs < HS; ++hs)
+            close_prev<CW>(sh.rsum[rb], dw, dh + 4 * hs, mnew_prev[hs], alpha_prev[hs],
+                           beta_prev[hs], k_prev[hs], m_h[hs], l_h[hs]);
         }
         // P.V of the tile decided kLag iterations ago
         if (n >= kLag) {
@@ -443,8 +464,9 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, 1)
             const bool vgot = mbar_wait_warp(&sh.v_full[vst], (vc / NV) & 1, ast, 12);
             // rescale: thread's accumulator columns are heads (lane&3)*2 + {0,1}
             const int h0 = (lane & 3) * 2;
-            const float a0 = (h0 < 4) ? sh.alpha[slot2][h0] : 1.f;
-            const float a1 = (h0 + 1 < 4) ? sh.alpha[slot2][h0 + 1] : 1.f;
+            // (one head slot: heads 4..7 are padding, alpha 1 and beta 0)
+            const float a0 = (HS == 1 && h0 >= 4) ? 1.f : sh.alpha[slot2][h0];
+            const float a1 = (HS == 1 && h0 + 1 >= 4) ? 1.f : sh.alpha[slot2][h0 + 1];
 #pragma unroll
             for (int mb = 0; mb < MB; ++mb) {
               acc[mb][0] *= a0; acc[mb][1] *= a1; acc[mb][2] *= a0; acc[mb][3] *= a1;
@@ -454,7 +476,7 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, 1)
 #pragma unroll
             for (int ks = 0; ks < (vgot ? kTile / 16 : 0); ++ks) {
               // P of key segment ks / KB, scaled to the tile's new maximum
-              const float bt = (hh < 4) ? sh.beta[slot2][ks / KB][hh] : 0.f;
+              const float bt = (HS == 1 && hh >= 4) ? 0.f : sh.beta[slot2][ks / KB][hh];
               const int kk = ks * 16 + (lane & 3) * 2;
               const float2 p0 = *reinterpret_cast<const float2*>(&sh.P[slot2][hh][kk]);
               const float2 p1 = *reinterpret_cast<const float2*>(&sh.P[slot2][hh][kk + 8]);
@@ -481,12 +503,16 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, 1)
       n_glob += nt;
       named_bar_sync(1, NT);
       if (*ast.flag) { ok = false; break; }
-      // this split's normalised output o_s = acc / l and z_s = (m + log2 l) ln 2; the
-      // state of head h sits in lanes 8h .. 8h+7
+      // this split's normalised output o_s = acc / l and z_s = (m + log2 l) ln 2
       {
         const int h0 = (lane & 3) * 2;
-        const float la = __shfl_sync(0xffffffffu, l_h, (h0 & 3) * 8);
-        const float lb = __shfl_sync(0xffffffffu, l_h, ((h0 + 1) & 3) * 8);
+        // head h's state sits in slot h / 4 of lanes 8 (h % 4) .. 8 (h % 4) + 7
+        const float l0a = __shfl_sync(0xffffffffu, l_h[0], (h0 & 3) * 8);
+        const float l1a = __shfl_sync(0xffffffffu, l_h[1], (h0 & 3) * 8);
+        const float l0b = __shfl_sync(0xffffffffu, l_h[0], ((h0 + 1) & 3) * 8);
+        const float l1b = __shfl_sync(0xffffffffu, l_h[1], ((h0 + 1) & 3) * 8);
+        const float la = (HS == 1 || h0 < 4) ? l0a : l1a;
+        const float lb = (HS == 1 || h0 + 1 < 4) ? l0b : l1b;
 #pragma unroll
         for (int mb = 0; mb < MB; ++mb)
 #pragma unroll
@@ -497,9 +523,11 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, 1)
               p.part_o[((static_cast<size_t>(b) * p.H + g * G + hh) * p.S + s) * D + dd] =
                   acc[mb][e] / ((e & 1) ? lb : la);
           }
-        if (warp == 0 && dw == 0 && dh < G)
-          p.part_z[(static_cast<size_t>(b) * p.H + g * G + dh) * p.S + s] =
-              (m_h + __log2f(l_h)) * kLn2;
+#pragma unroll
+        for (int hs = 0; hs < HS; ++hs)
+          if (warp == 0 && dw == 0 && dh + 4 * hs < G)
+            p.part_z[(static_cast<size_t>(b) * p.H + g * G + dh + 4 * hs) * p.S + s] =
+                (m_h[hs] + __log2f(l_h[hs])) * kLn2;
       }
       // last CTA of this (b, g) merges the splits
       named_bar_sync(1, NT);
@@ -559,10 +587,10 @@ mala_status fp32_decode(const float* q, const float* K, const float* V, float* O
                         int B, int H, int Hkv, int Nk, int d, float scale, float tau, int S,
                         bool screen, uint8_t* ws, uint8_t* tile_mask, cudaStream_t stream);
 
-template <int D, bool kScreen>
+template <int D, bool kScreen, int HS>
 static cudaError_t launch_decode(const CUtensorMap& tk, const CUtensorMap& tv,
                                  const DecParams& p, int grid, cudaStream_t stream) {
-  auto kern = mala_decode_kernel<D, kScreen>;
+  auto kern = mala_decode_kernel<D, kScreen, HS>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        DecCfg<D>::SMEM);
   if (e != cudaSuccess) return e;
@@ -582,7 +610,7 @@ mala_status decode_dispatch(const void* q, const void* K, const void* V, void* O
     return fp32_decode(static_cast<const float*>(q), static_cast<const float*>(K),
                        static_cast<const float*>(V), static_cast<float*>(O), LSE, B, H, Hkv, Nk,
                        d, scale, tau, num_splits, screen, ws, tile_mask, stream);
-  if (H / Hkv > 4) return MALA_ERR_UNSUPPORTED;  // the kernel packs up to 4 heads per group
+  if (H / Hkv > 8) return MALA_ERR_UNSUPPORTED;  // the kernel packs up to 8 heads per group
   CUtensorMap tk, tv;
   if (!make_tile_map(&tk, K, d, Hkv, Nk, B) || !make_tile_map(&tv, V, d, Hkv, Nk, B))
     return MALA_ERR_CUDA;
@@ -609,12 +637,17 @@ mala_status decode_dispatch(const void* q, const void* K, const void* V, void* O
     return MALA_ERR_CUDA;
   const int grid = p.n_units < sm_count() ? p.n_units : sm_count();
   cudaError_t e;
+  const bool wide = p.G > 4;
   if (d == 128)
-    e = screen ? launch_decode<128, true>(tk, tv, p, grid, stream)
-               : launch_decode<128, false>(tk, tv, p, grid, stream);
+    e = screen ? (wide ? launch_decode<128, true, 2>(tk, tv, p, grid, stream)
+                       : launch_decode<128, true, 1>(tk, tv, p, grid, stream))
+               : (wide ? launch_decode<128, false, 2>(tk, tv, p, grid, stream)
+                       : launch_decode<128, false, 1>(tk, tv, p, grid, stream));
   else
-    e = screen ? launch_decode<64, true>(tk, tv, p, grid, stream)
-               : launch_decode<64, false>(tk, tv, p, grid, stream);
+    e = screen ? (wide ? launch_decode<64, true, 2>(tk, tv, p, grid, stream)
+                       : launch_decode<64, true, 1>(tk, tv, p, grid, stream))
+               : (wide ? launch_decode<64, false, 2>(tk, tv, p, grid, stream)
+                       : launch_decode<64, false, 1>(tk, tv, p, grid, stream));
   return e == cudaSuccess ? MALA_OK : MALA_ERR_CUDA;
 }
 

@@ -120,3 +120,21 @@ def test_heavy128k_full(orc, mala):
     mask = check_decode(orc, mala, inp, w.scale, 1.0, S)
     group = mask.reshape(w.B, w.H_kv, w.H // w.H_kv, -1).max(axis=2)
     assert group.mean() < 0.35
+
+
+@pytest.mark.parametrize("tau", [0.0, 1.0])
+@pytest.mark.parametrize("shape", [(2, 16, 2, 3000, 128), (1, 24, 4, 1000, 64), (1, 5, 1, 700, 128)])
+def test_decode_large_groups(orc, mala, shape, tau):
+    """Groups of 5..8 query heads per KV head (e.g. 64 query / 8 KV heads)."""
+    w, inp = _planted(*shape, seed=31)
+    mask = check_decode(orc, mala, inp, w.scale, tau, 3)
+    if tau > 0 and shape[3] >= 1000:
+        assert (mask == 0).any()
+
+
+def test_decode_heavy_group8(orc, mala):
+    w = synth.Workload("adhoc_heavy8", 1, 16, 2, 8192, 128, "bf16", "heavy", 25, decode=True)
+    inp = synth.make_decode(w)
+    mask = check_decode(orc, mala, inp, w.scale, 1.0, 4)
+    group = mask.reshape(w.B, w.H_kv, w.H // w.H_kv, -1).max(axis=2)
+    assert group.mean() < 0.5
