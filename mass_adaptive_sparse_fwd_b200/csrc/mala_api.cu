@@ -329,6 +329,8 @@ mala_status mala_fwd_varlen(const void* Q, const void* K, const void* V, void* O
     return MALA_ERR_INVALID_ARG;
   const size_t need = mala_fwd_varlen_workspace_bytes(cu_seqlens_q, n_seqs, H, H_kv, d, dtype);
   if (workspace_bytes < need) return MALA_ERR_WORKSPACE;
+  if (static_cast<long long>(tab.size()) * H_kv * ((H / H_kv + 1) / 2) > (1ll << 30))
+    return MALA_ERR_UNSUPPORTED;  // unit count must fit the scheduler's 32-bit counter
   // heaviest first: the blocks with the most key tiles
   auto weight = [](const VarlenBlock& e) {
     return (e.off + std::min(e.i * kTile + kTile - 1, e.L - 1)) / kTile + 1;

@@ -261,8 +261,8 @@ def make_decode(w: Workload, Nk: int | None = None, B: int | None = None) -> dic
     elif w.structure == "heavy":
         # one heavy hitter shared by the group in every 8th key tile (key 64 of tiles
         # 7, 15, 23, ...): k = 28 u + 0.1 N(0, 1), u = the sum of the group's unit query
-        # directions, so each head scores it near 28 (|q_h| ~ sqrt(d), nearly orthogonal
-        # query directions) against ~N(0, 1) for the other keys
+        # directions, so each head scores it near 28 (17..33 over heads: |q_h| ~ sqrt(d),
+        # nearly orthogonal query directions) against ~N(0, 1) for the other keys
         for b in range(B):
             for g in range(Hkv):
                 qg = q[b, g * G:(g + 1) * G].astype(np.float64)

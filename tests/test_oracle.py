@@ -684,3 +684,41 @@ def test_prefill_units_match_full(orc):
         rows = slice(i * 16, min(50, (i + 1) * 16))
         np.testing.assert_array_equal(part[0][b, rows, h], full[0][b, rows, h])
         np.testing.assert_array_equal(part[2][b, h, i], full[2][b, h, i])
+
+
+@pytest.mark.parametrize("name", ["sinkband32k", "prevtok32k", "prevvar8k", "mixed8k"])
+def test_synth_training_structures_deterministic_and_bf16(name):
+    w = synth.WORKLOADS[name]
+    a = synth.make_training(w, L=384)
+    b = synth.make_training(w, L=384)
+    for k in a:
+        np.testing.assert_array_equal(a[k], b[k])
+    for k in ("Q", "K", "V"):
+        np.testing.assert_array_equal(synth.round_bf16(a[k]), a[k])
+        assert np.isfinite(a[k]).all()
+
+
+@pytest.mark.parametrize("name", ["decode128k", "heavy128k"])
+def test_synth_decode_structures_deterministic_and_bf16(name):
+    w = synth.WORKLOADS[name]
+    a = synth.make_decode(w, Nk=2048, B=1)
+    b = synth.make_decode(w, Nk=2048, B=1)
+    for k in a:
+        np.testing.assert_array_equal(a[k], b[k])
+        np.testing.assert_array_equal(synth.round_bf16(a[k]), a[k])
+
+
+def test_heavy_hitters_dominate_their_split(orc):
+    """The heavy128k recipe's claim: every 8th key tile holds a key that every head of the
+    group scores more than log(N_k / tau) = log(131072) ~ 11.8 above every other key, so a
+    split's tiles after its first heavy hitter fall below tau / N_k."""
+    w = synth.WORKLOADS["heavy128k"]
+    d = synth.make_decode(w, Nk=4096, B=1)
+    G = w.H // w.H_kv
+    q = d["q"][0].astype(np.float64)
+    K = d["K"][0].astype(np.float64)
+    for h in range(w.H):
+        s = K[:, h // G] @ q[h] * w.scale
+        heavy = s[7 * 128 + 64::8 * 128]
+        rest = np.delete(s, np.arange(7 * 128 + 64, 4096, 8 * 128))
+        assert heavy.min() > rest.max() + math.log(131072)
