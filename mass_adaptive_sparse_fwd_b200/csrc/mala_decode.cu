@@ -17,10 +17,15 @@
 //               at least one head of the group retains it.
 //   warps 0..CW-1  consumers (CW = 8 for d = 128, two per SM sub-partition, so one
 //               warp's dependent mma / shuffle / barrier chain hides another's):
-//               scores S = K_t q_g^T (mma.sync m16n8k16, heads padded to
-//               8 as the N dimension), per-head tile maxima, retention test, online
-//               softmax state and P_t; the P.V product of tile t is done LAG tiles
-//               later, when its V has had time to arrive.
+//               scores S = K_t q_g^T (mma.sync m16n8k16, heads padded to 8 as the
+//               N dimension) and per-warp maxima; one barrier per tile; then every
+//               warp takes the same per-head decision, lane-distributed, forms P_t
+//               against its own maxima only for kept tiles, and does the P.V product
+//               of tile t kLag tiles later, when its V has had time to arrive.  The
+//               row sums of a tile ride on the next tile's barrier, where they close
+//               its normaliser update before the next test.
+// Groups of up to 4 query heads run with one head slot per decision lane, groups of
+// 5..8 with two (template parameter HS).
 // The contraction per tile is tiny (128 keys x 128 dims x G heads) and the kernel is
 // bandwidth bound, so it uses warp-level mma.sync rather than tcgen05 / TMEM.
 

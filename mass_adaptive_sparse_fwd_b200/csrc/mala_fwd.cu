@@ -10,7 +10,9 @@
 // position down to 0 (diagonal first).  For chunked prefill (§2.3: the forward serves
 // inference prefill) the L query rows are the last L of Lk key positions: row q sits at
 // position off + q, off = Lk - L, attends to keys <= its position and has L_q = off + q + 1;
-// with off = 0 this is the ordinary causal forward.
+// with off = 0 this is the ordinary causal forward.  A packed batch of sequences of
+// different lengths (varlen) gives every unit its own sequence's row bases, length and
+// offset through a host-built table (FwdParams::vtab).
 //
 // Warp roles (384 threads):
 //   warp 0      TMA producer: Q of both slots, then K_j and V_j per key block into a
