@@ -328,7 +328,10 @@ def run_mala(args, dist: Dist):
             err = mala.read_device_error(ws)
             if err:
                 raise RuntimeError(f"device error word 0x{err:x}")
-        return {"step_ms": total, "fwd_ms": fwd, "bwd_ms": bwd, "decode_ms": dcd, "clocks": clk}
+        med = {"fwd_bwd_ms": statistics.median(e[0].elapsed_time(e[2]) for e in evs),
+               "decode_us": 1e3 * statistics.median(e[2].elapsed_time(e[3]) for e in evs)}
+        return {"step_ms": total, "fwd_ms": fwd, "bwd_ms": bwd, "decode_ms": dcd, "clocks": clk,
+                "median": med}
 
     clocks = ClockSampler(torch.cuda.current_device()) if dist.rank == 0 else None
     res = timed(TAU, clocks)
@@ -648,6 +651,7 @@ def run_mala(args, dist: Dist):
             "metric": METRIC, "value": step_fb, "unit": "ms", "n_gpus": dist.world,
             "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": res["step_ms"], "higher_is_better": False, "scaling": "weak",
+            "median": res["median"],  # per-step medians on rank 0 (value and the rest: means)
             "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded generator; states stand in for real model states)",
             "config": {"workload": f"{args.train} fwd+bwd (B={wt.B},H={wt.H},H_kv={wt.H_kv},"
