@@ -432,6 +432,7 @@ mala_status mala_decode(const void* q, const void* Kc, const void* Vc, void* O, 
   if (num_splits == 0) num_splits = decode_auto_splits(B, H_kv, Nk);
   if (num_splits < 1 || num_splits > T) return MALA_ERR_INVALID_ARG;
   if (dtype == MALA_BF16 && d != 64 && d != 128) return MALA_ERR_UNSUPPORTED;
+  if (dtype == MALA_BF16 && H / H_kv > 8) return MALA_ERR_UNSUPPORTED;  // up to 8 per group
   if (dtype == MALA_FP32 && d > 128) return MALA_ERR_UNSUPPORTED;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const size_t need = decode_workspace_bytes(B, H, H_kv, Nk, d, dtype, num_splits);

@@ -76,6 +76,7 @@ extern "C" mala_status mala_decode_noalloc(const void* q, const void* Kc, const 
   if (num_splits == 0) num_splits = decode_auto_splits(B, H_kv, Nk);
   if (num_splits < 1 || num_splits > T) return MALA_ERR_INVALID_ARG;
   if (dtype == MALA_BF16 && d != 64 && d != 128) return MALA_ERR_UNSUPPORTED;
+  if (dtype == MALA_BF16 && H / H_kv > 8) return MALA_ERR_UNSUPPORTED;  // up to 8 per group
   if (dtype == MALA_FP32 && d > 128) return MALA_ERR_UNSUPPORTED;
   const size_t need = decode_workspace_bytes(B, H, H_kv, Nk, d, dtype, num_splits);
   if (need > MALA_DECODE_NOALLOC_SCRATCH_BYTES) return MALA_ERR_WORKSPACE;

@@ -85,6 +85,12 @@ def test_invalid_arguments_are_rejected_before_any_launch(lib):
     # backward: bad dtype code
     assert L.mala_bwd(vp(), vp(), vp(), vp(), vp(), vp(), vp(), vp(), vp(), 1, 4, 2, 128, 128, 7,
                       0.1, 1.0, 0, None, 0, None, None) == 1
+    # decode: a group of more than 8 query heads per KV head on the bf16 path
+    assert L.mala_decode(vp(), vp(), vp(), vp(), vp(), 1, 18, 2, 256, 128, 0, 0.1, 1.0, 1, 0,
+                         vp(), 1 << 20, None, None) == 2
+    # prefill: more queries than keys
+    assert L.mala_fwd_prefill(vp(), vp(), vp(), vp(), vp(), 1, 4, 2, 300, 200, 128, 0, 0.1, 1.0,
+                              0, None, 0, None, None) == 1
     # statistics need a workspace and an output
     assert L.mala_get_stats(None, None, None) == 1
     # packed batches: offsets must start at 0 and every sequence needs N_k >= N_q
