@@ -39,6 +39,9 @@ TRAIN = "sinkband32k"  # --train sinkband128k times the 128K one-GPU training sh
 SKIP_TRAIN = "prevtok32k"  # concentrated states for the skip-regime block
 SKIP_DECODE = "heavy128k"  # KV cache with a heavy hitter in every 8th key tile
 DECODE = "decode128k"
+# the split count mala_decode_num_splits gives the decode workload (a host test checks it);
+# the reference arm, which does not load the library, runs its oracle decode with it
+DECODE_SPLITS = 9
 TAU = 1.0
 KERNELS_PER_STEP = 5  # fwd 1, bwd 3 (D preprocess, main, dQ convert), decode 1
 
@@ -238,7 +241,7 @@ def run_reference(args, dist: Dist):
     wt, wd = synth.WORKLOADS[TRAIN], synth.WORKLOADS[DECODE]
     train = synth.make_training(wt)
     dec = synth.make_decode(wd)
-    S = 37
+    S = DECODE_SPLITS
     vals = []
     for s in range(args.warmup + args.steps):
         ms, spent, desc = oracle_sample(wt, wd, train, dec, S, small=True)

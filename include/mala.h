@@ -200,7 +200,11 @@ size_t mala_bwd_workspace_bytes(int B, int H, int H_kv, int L, int d, int dtype)
 size_t mala_decode_workspace_bytes(int B, int H, int H_kv, int Nk, int d, int dtype,
                                    int num_splits);
 
-/* The split count used when mala_decode is given num_splits = 0 (deterministic). */
+/* The split count used when mala_decode is given num_splits = 0 (deterministic, host
+ * only, no device query).  Among the counts that give at most two waves of units
+ * (b, KV head, split) over 148 persistent CTAs, it takes the S that minimises
+ * waves x (ceil(T / S) + 10): a CTA's time is its key tiles plus a fixed cost of about
+ * ten tiles per unit.  Ties go to fewer splits.  Returns 0 for invalid shapes. */
 int mala_decode_num_splits(int B, int H, int H_kv, int Nk);
 
 /* Reads the device error word of a workspace (synchronises `stream`).  *out receives

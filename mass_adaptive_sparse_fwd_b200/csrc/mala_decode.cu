@@ -570,15 +570,31 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, 1)
 }  // namespace
 
 int decode_auto_splits(int B, int Hkv, int Nk) {
-  // about eight persistent-CTA waves on a 148-SM B200, at least 8 key tiles per split
+  // A persistent CTA (one per SM of a 148-SM B200) takes units (b, g, split) round-robin,
+  // so its time is about waves x (key tiles per split + a fixed cost per unit: the q load,
+  // the pipeline fill and drain, the partial write and the ticket), the fixed cost being
+  // worth about 10 tiles at the HBM rate.  One SM alone streams K and V at about 1/148 of
+  // the HBM rate, so a single wave of fewer CTAs is not bandwidth-starved beyond its tile
+  // count.  The rule takes the split count S <= T of at most two waves that minimises
+  // ceil(B Hkv S / 148) (ceil(T / S) + 10); ties go to fewer splits (fewer partials to
+  // merge).
+  constexpr int kSMs = 148, kUnitCostTiles = 10;
   const int T = (Nk + kTile - 1) / kTile;
   const int bg = B * Hkv;
-  int s = (8 * 148 + bg / 2) / bg;
-  const int cap = T / 8 > 1 ? T / 8 : 1;
-  if (s > cap) s = cap;
-  if (s < 1) s = 1;
-  if (s > T) s = T;
-  return s;
+  int smax = (2 * kSMs) / bg;
+  if (smax > T) smax = T;
+  if (smax < 1) smax = 1;
+  int best_s = 1;
+  long long best_cost = -1;
+  for (int s = 1; s <= smax; ++s) {
+    const long long waves = (static_cast<long long>(bg) * s + kSMs - 1) / kSMs;
+    const long long cost = waves * ((T + s - 1) / s + kUnitCostTiles);
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best_s = s;
+    }
+  }
+  return best_s;
 }
 
 size_t decode_workspace_bytes(int B, int H, int Hkv, int Nk, int d, int dtype, int S) {

@@ -117,6 +117,27 @@ def test_workspace_sizes_and_split_rule(lib):
     assert lib.decode_workspace_bytes(1, 4, 2, 256, 128, 0, 5) == 0  # 5 splits > 2 tiles
 
 
+@pytest.mark.parametrize("shape,expect", [
+    ((4, 32, 8, 131072), 9),    # 288 units: two full waves of 228 tiles per CTA
+    ((4, 32, 8, 32768), 4),     # one wave of 128 CTAs
+    ((1, 32, 8, 131072), 18),   # one wave of 144 CTAs
+    ((8, 32, 8, 32768), 2),
+    ((1, 8, 1, 524288), 147),
+    ((64, 32, 8, 131072), 1),   # 512 (b, g) pairs: one split each
+    ((1, 4, 1, 300), 3),        # one tile per split
+])
+def test_split_rule_values(lib, shape, expect):
+    """The split rule: at most two waves of 148 persistent CTAs, minimising
+    waves x (tiles per split + 10), fewer splits on ties."""
+    assert lib.decode_num_splits(*shape) == expect
+
+
+def test_bench_reference_split_count(lib):
+    import bench
+    w = bench.synth.WORKLOADS[bench.DECODE]
+    assert lib.decode_num_splits(w.B, w.H, w.H_kv, w.L) == bench.DECODE_SPLITS
+
+
 def test_bench_accounting():
     sys.path.insert(0, ROOT)
     import bench
