@@ -161,7 +161,10 @@ mala_status mala_decode(const void* q, const void* Kc, const void* Vc, void* O, 
  *   Same arguments and results as mala_decode without the workspace: the scratch comes
  *   from a fixed array of MALA_DECODE_NOALLOC_SCRATCH_BYTES compiled into the library,
  *   which every GPU that loads the library holds until the process exits.  Calls whose
- *   mala_decode_workspace_bytes() exceeds that size return MALA_ERR_WORKSPACE.
+ *   mala_decode_workspace_bytes() exceeds that size return MALA_ERR_WORKSPACE.  With
+ *   num_splits = 0 the split rule keeps B * H_kv * S <= 296 whenever B * H_kv <= 296, so
+ *   the scratch is at most 296 * (H / H_kv) * (d + 1) * 4 bytes plus a small header:
+ *   every bf16 decode (groups of up to 8) of such a batch fits.
  *   The first call on a device looks up the array's device address (once per device,
  *   with that device current); make that first call before any stream capture.
  *   All calls on a device share the array: calls whose work overlaps on the GPU (two

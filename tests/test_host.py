@@ -132,6 +132,23 @@ def test_split_rule_values(lib, shape, expect):
     assert lib.decode_num_splits(*shape) == expect
 
 
+def test_auto_splits_fit_the_noalloc_scratch(lib):
+    """With num_splits = 0 a bf16 decode (groups of up to 8) of a batch with
+    B * H_kv <= 296 needs at most 296 units, so its scratch fits the in-library array of
+    mala_decode_noalloc (4 MiB)."""
+    for B in (1, 2, 3, 4, 8, 16, 37, 64):
+        for Hkv in (1, 2, 4, 8):
+            if B * Hkv > 296:
+                continue
+            for Nk in (1, 127, 129, 1000, 8192, 65536, 131072, 1 << 20):
+                for d in (64, 128):
+                    S = lib.decode_num_splits(B, 8 * Hkv, Hkv, Nk)
+                    assert 1 <= S and B * Hkv * S <= 296
+                    assert S <= -(-Nk // 128)
+                    ws = lib.decode_workspace_bytes(B, 8 * Hkv, Hkv, Nk, d, 0, 0)
+                    assert 0 < ws <= 4 << 20
+
+
 def test_bench_reference_split_count(lib):
     import bench
     w = bench.synth.WORKLOADS[bench.DECODE]
