@@ -111,7 +111,9 @@ mala_status mala_fwd_prefill(const void* Q, const void* K, const void* V, void* 
  *   with cudaMemcpyAsync, so the call waits for earlier work on `stream` before it
  *   returns (pageable staging) and cannot be captured in a CUDA graph.  No tile_mask;
  *   mala_get_stats reports the call's tiles.  Each sequence's results equal those of
- *   mala_fwd_prefill on that sequence alone.
+ *   mala_fwd_prefill on that sequence alone.  A batch with no query rows at all returns
+ *   MALA_OK after the host checks, with no CUDA call (the workspace, statistics included,
+ *   is left as it was).
  */
 size_t mala_fwd_varlen_workspace_bytes(const int* cu_seqlens_q, int n_seqs, int H, int H_kv,
                                        int d, int dtype);
