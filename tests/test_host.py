@@ -100,6 +100,9 @@ def test_invalid_arguments_are_rejected_before_any_launch(lib):
     assert L.mala_fwd_varlen(vp(), vp(), vp(), vp(), vp(), ia([0, 10]), ia([0, 5]), *args) == 1
     assert L.mala_fwd_varlen_workspace_bytes(ia([0, 300, 300, 557]), 3, 4, 2, 128, 0) == \
         256 + (3 + 0 + 3) * 32
+    # a batch with no query rows is done after the host checks (no CUDA call)
+    assert L.mala_fwd_varlen(vp(), vp(), vp(), vp(), vp(), ia([0, 0, 0]), ia([0, 5, 7]), 2,
+                             *args[1:]) == 0
     # workspace too small (checked before any CUDA call)
     assert L.mala_fwd(vp(), vp(), vp(), vp(), vp(), 1, 4, 2, 128, 128, 0, 0.1, 1.0, 0, vp(), 8,
                       None, None) == 5
