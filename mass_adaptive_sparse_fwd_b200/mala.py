@@ -119,6 +119,58 @@ def _check(fn: str, status: int):
         raise MalaError(fn, status)
 
 
+# The C ABI receives bare pointers and sizes, so a tensor whose shape, dtype or layout
+# disagrees with the sizes passed next to it would send the kernels past its allocation.
+# Every entry point below checks its tensors against the layouts of include/mala.h first
+# (shape, dtype, contiguity, one device), and only then requires that device to be CUDA.
+
+
+def _need(fn, name, t, shape, dtype, device):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{fn}: {name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{fn}: {name} has dtype {t.dtype}, expected {dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{fn}: {name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{fn}: {name} must be contiguous")
+    if t.device != device:
+        raise ValueError(f"{fn}: {name} is on {t.device}, the call's tensors on {device}")
+
+
+def _need_buffer(fn, name, t, min_numel, dtype, device):
+    """An optional flat buffer (tile mask): at least min_numel elements of dtype."""
+    if t is None:
+        return
+    if not isinstance(t, torch.Tensor) or t.dtype != dtype:
+        raise TypeError(f"{fn}: {name} must be a {dtype} tensor")
+    if t.numel() < min_numel:
+        raise ValueError(f"{fn}: {name} holds {t.numel()} elements, needs {min_numel}")
+    if not t.is_contiguous() or t.device != device:
+        raise ValueError(f"{fn}: {name} must be contiguous and on {device}")
+
+
+def _workspace_bytes(fn, workspace, device) -> int:
+    if workspace is None:
+        return 0
+    if not isinstance(workspace, torch.Tensor) or not workspace.is_contiguous() or \
+            workspace.device != device:
+        raise ValueError(f"{fn}: workspace must be a contiguous tensor on {device}")
+    return workspace.numel() * workspace.element_size()
+
+
+def _need_cuda(fn, device):
+    if device.type != "cuda":
+        raise ValueError(f"{fn}: tensors must be on a CUDA device, got {device}")
+
+
+def _qkv_dtype(fn, Q) -> torch.dtype:
+    if not isinstance(Q, torch.Tensor):
+        raise TypeError(f"{fn}: Q must be a torch.Tensor")
+    _dtype_code(Q)  # bf16 or fp32
+    return Q.dtype
+
+
 def n_tiles(n: int) -> int:
     return (n + TILE - 1) // TILE
 
@@ -148,13 +200,22 @@ def mala_fwd(Q, K, V, scale, tau, O=None, LSE=None, flags=0, workspace=None, til
              stream=None):
     """MALA forward through the C ABI.  Q [B,L,H,d], K/V [B,L,H_kv,d] (bf16 or fp32,
     contiguous, on the GPU).  Returns (O, LSE)."""
+    fn, dt = "mala_fwd", _qkv_dtype("mala_fwd", Q)
     B, L, H, d = Q.shape
-    H_kv = K.shape[2]
+    H_kv = K.shape[2] if isinstance(K, torch.Tensor) and K.dim() == 4 else -1
+    dev = Q.device
+    _need(fn, "Q", Q, (B, L, H, d), dt, dev)
+    _need(fn, "K", K, (B, L, H_kv, d), dt, dev)
+    _need(fn, "V", V, (B, L, H_kv, d), dt, dev)
     if O is None:
         O = torch.empty_like(Q)
     if LSE is None:
-        LSE = torch.empty((B, H, L), dtype=torch.float32, device=Q.device)
-    ws_bytes = 0 if workspace is None else workspace.numel()
+        LSE = torch.empty((B, H, L), dtype=torch.float32, device=dev)
+    _need(fn, "O", O, (B, L, H, d), dt, dev)
+    _need(fn, "LSE", LSE, (B, H, L), torch.float32, dev)
+    _need_buffer(fn, "tile_mask", tile_mask, B * H * n_tiles(L) ** 2, torch.uint8, dev)
+    ws_bytes = _workspace_bytes(fn, workspace, dev)
+    _need_cuda(fn, dev)
     st = _lib.mala_fwd(_ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(LSE), B, H, H_kv, L, d,
                        _dtype_code(Q), float(scale), float(tau), flags, _ptr(workspace), ws_bytes,
                        _ptr(tile_mask), _stream(stream))
@@ -167,13 +228,24 @@ def mala_fwd_prefill(Q, K, V, scale, tau, O=None, LSE=None, flags=0, workspace=N
     """Forward of a prefill chunk through the C ABI: Q [B,N_q,H,d] are the last N_q
     positions of the sequence whose keys K/V [B,N_k,H_kv,d] (N_k >= N_q) include them.
     Returns (O [B,N_q,H,d], LSE [B,H,N_q])."""
+    fn, dt = "mala_fwd_prefill", _qkv_dtype("mala_fwd_prefill", Q)
     B, Nq, H, d = Q.shape
-    Nk, H_kv = K.shape[1], K.shape[2]
+    Nk, H_kv = (K.shape[1], K.shape[2]) if isinstance(K, torch.Tensor) and K.dim() == 4 \
+        else (-1, -1)
+    dev = Q.device
+    _need(fn, "K", K, (B, Nk, H_kv, d), dt, dev)
+    _need(fn, "V", V, (B, Nk, H_kv, d), dt, dev)
+    _need(fn, "Q", Q, (B, Nq, H, d), dt, dev)
     if O is None:
         O = torch.empty_like(Q)
     if LSE is None:
-        LSE = torch.empty((B, H, Nq), dtype=torch.float32, device=Q.device)
-    ws_bytes = 0 if workspace is None else workspace.numel()
+        LSE = torch.empty((B, H, Nq), dtype=torch.float32, device=dev)
+    _need(fn, "O", O, (B, Nq, H, d), dt, dev)
+    _need(fn, "LSE", LSE, (B, H, Nq), torch.float32, dev)
+    _need_buffer(fn, "tile_mask", tile_mask, B * H * n_tiles(Nq) * n_tiles(Nk), torch.uint8,
+                 dev)
+    ws_bytes = _workspace_bytes(fn, workspace, dev)
+    _need_cuda(fn, dev)
     st = _lib.mala_fwd_prefill(_ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(LSE), B, H, H_kv, Nq, Nk,
                                d, _dtype_code(Q), float(scale), float(tau), flags,
                                _ptr(workspace), ws_bytes, _ptr(tile_mask), _stream(stream))
@@ -196,19 +268,35 @@ def mala_fwd_varlen(Q, K, V, cu_seqlens_q, cu_seqlens_k, scale, tau, O=None, LSE
     """Forward of a packed batch through the C ABI: Q [total_q,H,d], K/V [total_k,H_kv,d];
     cu_seqlens_* are host sequences of n+1 offsets.  Returns (O [total_q,H,d],
     LSE [H,total_q])."""
+    fn, dt = "mala_fwd_varlen", _qkv_dtype("mala_fwd_varlen", Q)
     total_q, H, d = Q.shape
-    H_kv = K.shape[1]
+    H_kv = K.shape[1] if isinstance(K, torch.Tensor) and K.dim() == 3 else -1
     n = len(cu_seqlens_q) - 1
+    if n < 1 or len(cu_seqlens_k) != n + 1:
+        raise ValueError(f"{fn}: cu_seqlens_q / cu_seqlens_k need the same n + 1 >= 2 offsets")
+    total_k = int(cu_seqlens_k[-1])
+    if int(cu_seqlens_q[-1]) != total_q:
+        raise ValueError(f"{fn}: cu_seqlens_q ends at {int(cu_seqlens_q[-1])}, Q has "
+                         f"{total_q} rows")
+    dev = Q.device
+    _need(fn, "Q", Q, (total_q, H, d), dt, dev)
+    _need(fn, "K", K, (total_k, H_kv, d), dt, dev)
+    _need(fn, "V", V, (total_k, H_kv, d), dt, dev)
     if O is None:
         O = torch.empty_like(Q)
     if LSE is None:
-        LSE = torch.empty((H, total_q), dtype=torch.float32, device=Q.device)
+        LSE = torch.empty((H, total_q), dtype=torch.float32, device=dev)
+    _need(fn, "O", O, (total_q, H, d), dt, dev)
+    _need(fn, "LSE", LSE, (H, total_q), torch.float32, dev)
     if workspace is None:
-        workspace = alloc_workspace(varlen_workspace_bytes(cu_seqlens_q, H, H_kv, d), Q.device)
+        _need_cuda(fn, dev)
+        workspace = alloc_workspace(varlen_workspace_bytes(cu_seqlens_q, H, H_kv, d), dev)
+    ws_bytes = _workspace_bytes(fn, workspace, dev)
+    _need_cuda(fn, dev)
     st = _lib.mala_fwd_varlen(_ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(LSE),
                               _int_array(cu_seqlens_q), _int_array(cu_seqlens_k), n, H, H_kv, d,
                               _dtype_code(Q), float(scale), float(tau), flags, _ptr(workspace),
-                              workspace.numel(), _stream(stream))
+                              ws_bytes, _stream(stream))
     _check("mala_fwd_varlen", st)
     return O, LSE
 
@@ -216,12 +304,25 @@ def mala_fwd_varlen(Q, K, V, cu_seqlens_q, cu_seqlens_k, scale, tau, O=None, LSE
 def mala_bwd(Q, K, V, O, LSE, dO, scale, tau, dQ=None, dK=None, dV=None, flags=0,
              workspace=None, tile_mask=None, stream=None):
     """MALA backward through the C ABI.  Returns (dQ, dK, dV)."""
+    fn, dt = "mala_bwd", _qkv_dtype("mala_bwd", Q)
     B, L, H, d = Q.shape
-    H_kv = K.shape[2]
+    H_kv = K.shape[2] if isinstance(K, torch.Tensor) and K.dim() == 4 else -1
+    dev = Q.device
+    _need(fn, "Q", Q, (B, L, H, d), dt, dev)
+    _need(fn, "K", K, (B, L, H_kv, d), dt, dev)
+    _need(fn, "V", V, (B, L, H_kv, d), dt, dev)
+    _need(fn, "O", O, (B, L, H, d), dt, dev)
+    _need(fn, "LSE", LSE, (B, H, L), torch.float32, dev)
+    _need(fn, "dO", dO, (B, L, H, d), dt, dev)
     dQ = torch.empty_like(Q) if dQ is None else dQ
     dK = torch.empty_like(K) if dK is None else dK
     dV = torch.empty_like(V) if dV is None else dV
-    ws_bytes = 0 if workspace is None else workspace.numel()
+    _need(fn, "dQ", dQ, (B, L, H, d), dt, dev)
+    _need(fn, "dK", dK, (B, L, H_kv, d), dt, dev)
+    _need(fn, "dV", dV, (B, L, H_kv, d), dt, dev)
+    _need_buffer(fn, "tile_mask", tile_mask, B * H * n_tiles(L) ** 2, torch.uint8, dev)
+    ws_bytes = _workspace_bytes(fn, workspace, dev)
+    _need_cuda(fn, dev)
     st = _lib.mala_bwd(_ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(LSE), _ptr(dO), _ptr(dQ), _ptr(dK),
                        _ptr(dV), B, H, H_kv, L, d, _dtype_code(Q), float(scale), float(tau), flags,
                        _ptr(workspace), ws_bytes, _ptr(tile_mask), _stream(stream))
@@ -229,15 +330,33 @@ def mala_bwd(Q, K, V, O, LSE, dO, scale, tau, dQ=None, dK=None, dV=None, flags=0
     return dQ, dK, dV
 
 
+def _decode_checks(fn, q, Kc, Vc, O, LSE, tile_mask):
+    dt = _qkv_dtype(fn, q)
+    B, H, d = q.shape
+    Nk, H_kv = (Kc.shape[1], Kc.shape[2]) if isinstance(Kc, torch.Tensor) and Kc.dim() == 4 \
+        else (-1, -1)
+    dev = q.device
+    _need(fn, "q", q, (B, H, d), dt, dev)
+    _need(fn, "Kc", Kc, (B, Nk, H_kv, d), dt, dev)
+    _need(fn, "Vc", Vc, (B, Nk, H_kv, d), dt, dev)
+    if O is not None:
+        _need(fn, "O", O, (B, H, d), dt, dev)
+    if LSE is not None:
+        _need(fn, "LSE", LSE, (B, H), torch.float32, dev)
+    _need_buffer(fn, "tile_mask", tile_mask, B * H * n_tiles(Nk), torch.uint8, dev)
+    return B, H, d, Nk, H_kv
+
+
 def mala_decode(q, Kc, Vc, scale, tau, num_splits=0, O=None, LSE=None, flags=0, workspace=None,
                 tile_mask=None, stream=None):
     """MALA split-KV decode through the C ABI.  q [B,H,d]; Kc/Vc [B,N_k,H_kv,d].
     Returns (O [B,H,d], LSE [B,H])."""
-    B, H, d = q.shape
-    Nk, H_kv = Kc.shape[1], Kc.shape[2]
+    fn = "mala_decode"
+    B, H, d, Nk, H_kv = _decode_checks(fn, q, Kc, Vc, O, LSE, tile_mask)
     O = torch.empty_like(q) if O is None else O
     LSE = torch.empty((B, H), dtype=torch.float32, device=q.device) if LSE is None else LSE
-    ws_bytes = 0 if workspace is None else workspace.numel()
+    ws_bytes = _workspace_bytes(fn, workspace, q.device)
+    _need_cuda(fn, q.device)
     st = _lib.mala_decode(_ptr(q), _ptr(Kc), _ptr(Vc), _ptr(O), _ptr(LSE), B, H, H_kv, Nk, d,
                           _dtype_code(q), float(scale), float(tau), int(num_splits), flags,
                           _ptr(workspace), ws_bytes, _ptr(tile_mask), _stream(stream))
@@ -251,10 +370,11 @@ def mala_decode_noalloc(q, Kc, Vc, scale, tau, num_splits=0, O=None, LSE=None, f
     array inside the library (for callers that may not allocate device memory on their
     hot path).  Calls on one device share that array, so they must not overlap on the
     GPU.  Returns (O [B,H,d], LSE [B,H])."""
-    B, H, d = q.shape
-    Nk, H_kv = Kc.shape[1], Kc.shape[2]
+    fn = "mala_decode_noalloc"
+    B, H, d, Nk, H_kv = _decode_checks(fn, q, Kc, Vc, O, LSE, tile_mask)
     O = torch.empty_like(q) if O is None else O
     LSE = torch.empty((B, H), dtype=torch.float32, device=q.device) if LSE is None else LSE
+    _need_cuda(fn, q.device)
     st = _lib.mala_decode_noalloc(_ptr(q), _ptr(Kc), _ptr(Vc), _ptr(O), _ptr(LSE), B, H, H_kv,
                                   Nk, d, _dtype_code(q), float(scale), float(tau),
                                   int(num_splits), flags, _ptr(tile_mask), _stream(stream))
