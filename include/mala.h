@@ -234,7 +234,8 @@ mala_status mala_set_wait_budget_ns(uint64_t ns);
 
 const char* mala_status_string(mala_status s);
 
-/* Library version: 200 = 0.2.0 (adds mala_fwd_prefill, mala_fwd_varlen, mala_get_stats). */
+/* Library version: 201 = 0.2.1 (0.2.0 added mala_fwd_prefill, mala_fwd_varlen and
+ * mala_get_stats; 0.2.1 changes the automatic decode split count, mala_decode_num_splits). */
 int mala_version(void);
 
 #ifdef __cplusplus

@@ -136,7 +136,7 @@ using namespace mala;
 
 extern "C" {
 
-int mala_version(void) { return 200; }
+int mala_version(void) { return 201; }
 
 const char* mala_status_string(mala_status s) {
   switch (s) {

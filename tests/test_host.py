@@ -52,7 +52,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 def test_version_and_status_strings(lib):
     L = lib.lib()
-    assert L.mala_version() == 200
+    assert L.mala_version() == 201
     assert L.mala_status_string(0) == b"ok"
     assert L.mala_status_string(4) == b"device wait timed out"
 
