@@ -232,10 +232,43 @@ mala_status mala_selftest_wait_timeout(void* workspace, uint64_t budget_ns, void
 /* Sets the wall-clock budget of every internal wait (default 2 s; test hook). */
 mala_status mala_set_wait_budget_ns(uint64_t ns);
 
+/*
+ * mala_set_debug - test hook that exports the margin of every retention test.
+ * The decisions are the threshold tests of "MassAlloc Attention" §2.2 Eq. (3) (forward),
+ * Eq. (4) (backward) and §2.4 (decode); this hook reports how far each tested tile was
+ * from its threshold, so that a caller can compare the decisions against an independent
+ * evaluation and see how close a disagreeing tile was.  The page has no API for it.
+ *   dbg->tile_margin: DEVICE float32 buffer with the layout of the call's tile_mask
+ *   ([B,H,T,Tk] for mala_fwd / mala_fwd_prefill, [B,H,T,T] for mala_bwd, [B,H,T] for
+ *   mala_decode); dbg->tile_margin_count: floats available in it.  Passing NULL, or a
+ *   NULL tile_margin, turns the hook off.  The setting belongs to the calling host
+ *   thread and stays until changed; mala_fwd_varlen and mala_decode_noalloc ignore it.
+ *   A call that needs more entries than tile_margin_count returns MALA_ERR_INVALID_ARG
+ *   before anything is launched.
+ *   Each call first fills its entries with the all-ones bit pattern (a NaN) and then
+ *   writes, for every tile whose test ran, the margin in natural-log units:
+ *     forward: max over the block's rows with a legal key of
+ *              max_k s_qk - log Z_q - log(tau / L_q), Z_q the running normaliser of the
+ *              tiles retained so far, +inf if some such row has Z_q = 0;
+ *     backward: max over the tile's legal entries of s_qk - LSE_q - log(tau / L_q);
+ *     decode:  max_k s_k - log Z - log(tau / N_k) per head, Z the split's running
+ *              normaliser, +inf on the first tile of a split.
+ *   The tile is retained exactly when its margin is >= 0.  Margins are written only when
+ *   the test runs (tau > 0 or MALA_FLAG_ALWAYS_TEST); other entries stay NaN.  The
+ *   kernels combine the forward and backward margins with float atomics, so a call with
+ *   the hook on runs slower.
+ */
+typedef struct {
+  float* tile_margin;
+  size_t tile_margin_count;
+} mala_debug;
+mala_status mala_set_debug(const mala_debug* dbg);
+
 const char* mala_status_string(mala_status s);
 
-/* Library version: 201 = 0.2.1 (0.2.0 added mala_fwd_prefill, mala_fwd_varlen and
- * mala_get_stats; 0.2.1 changes the automatic decode split count, mala_decode_num_splits). */
+/* Library version: 202 = 0.2.2 (0.2.0 added mala_fwd_prefill, mala_fwd_varlen and
+ * mala_get_stats; 0.2.1 changes the automatic decode split count, mala_decode_num_splits;
+ * 0.2.2 adds mala_set_debug). */
 int mala_version(void);
 
 #ifdef __cplusplus

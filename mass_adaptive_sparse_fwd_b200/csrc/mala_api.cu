@@ -21,18 +21,19 @@ cudaError_t launch_fwd_bf16(const CUtensorMap& tq, const CUtensorMap& tk, const 
 mala_status bwd_dispatch(const void* Q, const void* K, const void* V, const void* O,
                          const float* LSE, const void* dO, void* dQ, void* dK, void* dV, int B,
                          int H, int Hkv, int L, int d, int dtype, float scale, float tau,
-                         unsigned flags, uint8_t* ws, uint8_t* tile_mask, uint64_t budget_ns,
-                         cudaStream_t stream);
+                         unsigned flags, uint8_t* ws, uint8_t* tile_mask, float* tile_margin,
+                         uint64_t budget_ns, cudaStream_t stream);
 size_t bwd_workspace_bytes(int B, int H, int Hkv, int L, int d, int dtype);
 mala_status decode_dispatch(const void* q, const void* K, const void* V, void* O, float* LSE,
                             int B, int H, int Hkv, int Nk, int d, int dtype, float scale,
                             float tau, int num_splits, unsigned flags, uint8_t* ws,
-                            uint8_t* tile_mask, uint64_t budget_ns, cudaStream_t stream);
+                            uint8_t* tile_mask, float* tile_margin, uint64_t budget_ns,
+                            cudaStream_t stream);
 size_t decode_workspace_bytes(int B, int H, int Hkv, int Nk, int d, int dtype, int num_splits);
 int decode_auto_splits(int B, int Hkv, int Nk);
 mala_status fp32_fwd(const float* Q, const float* K, const float* V, float* O, float* LSE, int B,
                      int H, int Hkv, int L, int Lk, int d, float scale, float tau, bool screen,
-                     uint8_t* ws, uint8_t* tile_mask, cudaStream_t stream);
+                     uint8_t* ws, uint8_t* tile_mask, float* tile_margin, cudaStream_t stream);
 
 // ---------------------------------------------------------------------------- shared host helpers
 
@@ -80,6 +81,28 @@ int sm_count() {
 static uint64_t g_budget_ns = 2000000000ull;
 
 uint64_t wait_budget_ns() { return g_budget_ns; }
+
+// Debug margin buffer of the calling host thread (mala_set_debug).
+static thread_local float* t_margin = nullptr;
+static thread_local size_t t_margin_count = 0;
+
+// The margin buffer for a call that tests `entries` tiles: null when debugging is off.
+// `ok` turns false when the registered buffer is too small for the call.
+float* debug_margin(size_t entries, bool& ok) {
+  ok = true;
+  if (!t_margin) return nullptr;
+  if (t_margin_count < entries) {
+    ok = false;
+    return nullptr;
+  }
+  return t_margin;
+}
+
+// Fills the first `entries` margins with the all-ones bit pattern (a NaN): entries of
+// tiles that are not tested keep it, and the kernels' float max starts from it.
+bool debug_margin_clear(float* margin, size_t entries, cudaStream_t stream) {
+  return !margin || cudaMemsetAsync(margin, 0xff, entries * sizeof(float), stream) == cudaSuccess;
+}
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -136,7 +159,7 @@ using namespace mala;
 
 extern "C" {
 
-int mala_version(void) { return 201; }
+int mala_version(void) { return 202; }
 
 const char* mala_status_string(mala_status s) {
   switch (s) {
@@ -153,6 +176,19 @@ const char* mala_status_string(mala_status s) {
 mala_status mala_set_wait_budget_ns(uint64_t ns) {
   if (ns == 0) return MALA_ERR_INVALID_ARG;
   g_budget_ns = ns;
+  return MALA_OK;
+}
+
+mala_status mala_set_debug(const mala_debug* dbg) {
+  if (!dbg || !dbg->tile_margin) {
+    t_margin = nullptr;
+    t_margin_count = 0;
+    return MALA_OK;
+  }
+  if ((reinterpret_cast<uintptr_t>(dbg->tile_margin) & 3u) != 0 || dbg->tile_margin_count == 0)
+    return MALA_ERR_INVALID_ARG;
+  t_margin = dbg->tile_margin;
+  t_margin_count = dbg->tile_margin_count;
   return MALA_OK;
 }
 
@@ -220,6 +256,9 @@ mala_status run_fwd(const void* Q, const void* K, const void* V, void* O, float*
   const bool screen = (tau > 0.f) || (flags & MALA_FLAG_ALWAYS_TEST);
   const int T = (L + kTile - 1) / kTile;
   const int Tk = (Lk + kTile - 1) / kTile;
+  bool margin_ok = true;
+  float* margin = debug_margin(static_cast<size_t>(B) * H * T * Tk, margin_ok);
+  if (!margin_ok) return MALA_ERR_INVALID_ARG;
   if (dtype == MALA_FP32) {
     if (d > 128) return MALA_ERR_UNSUPPORTED;
     // this path needs no scratch; a caller's workspace only receives the call statistics
@@ -232,9 +271,10 @@ mala_status run_fwd(const void* Q, const void* K, const void* V, void* O, float*
           cudaSuccess)
         return MALA_ERR_CUDA;
     }
+    if (!debug_margin_clear(margin, static_cast<size_t>(B) * H * T * Tk, st)) return MALA_ERR_CUDA;
     return fp32_fwd(static_cast<const float*>(Q), static_cast<const float*>(K),
                     static_cast<const float*>(V), static_cast<float*>(O), LSE, B, H, H_kv, L, Lk,
-                    d, scale, tau, screen, ws, tile_mask, st);
+                    d, scale, tau, screen, ws, tile_mask, margin, st);
   }
   if (d != 64 && d != 128) return MALA_ERR_UNSUPPORTED;
   if ((long long)B * Lk > (1ll << 31) || (long long)B * H * T > (1ll << 30))
@@ -249,7 +289,8 @@ mala_status run_fwd(const void* Q, const void* K, const void* V, void* O, float*
   return with_workspace(workspace, workspace_bytes, need, st, [&](uint8_t* ws) -> mala_status {
     uint32_t* hdr = reinterpret_cast<uint32_t*>(ws);
     if (cudaMemsetAsync(hdr + kHdrSched0, 0, 3 * sizeof(uint32_t), st) != cudaSuccess ||
-        cudaMemsetAsync(ws + kStatsOffset, 0, 3 * sizeof(unsigned long long), st) != cudaSuccess)
+        cudaMemsetAsync(ws + kStatsOffset, 0, 3 * sizeof(unsigned long long), st) != cudaSuccess ||
+        !debug_margin_clear(margin, static_cast<size_t>(B) * H * T * Tk, st))
       return MALA_ERR_CUDA;
     FwdParams p;
     p.B = B; p.H = H; p.Hkv = H_kv; p.L = L; p.T = T; p.G = H / H_kv;
@@ -261,6 +302,7 @@ mala_status run_fwd(const void* Q, const void* K, const void* V, void* O, float*
     p.scale_log2 = scale * kLog2e;
     p.log2_tau = (tau > 0.f) ? std::log2(tau) : -INFINITY;
     p.O = O; p.LSE = LSE; p.tile_mask = tile_mask;
+    p.tile_margin = margin;
     p.err = hdr + kHdrError;
     p.sched = hdr + kHdrSched0;
     p.budget_ns = wait_budget_ns();
@@ -363,6 +405,7 @@ mala_status mala_fwd_varlen(const void* Q, const void* K, const void* V, void* O
   p.scale_log2 = scale * kLog2e;
   p.log2_tau = (tau > 0.f) ? std::log2(tau) : -INFINITY;
   p.O = O; p.LSE = LSE; p.tile_mask = nullptr;
+  p.tile_margin = nullptr;
   p.err = hdr + kHdrError;
   p.sched = hdr + kHdrSched0;
   p.budget_ns = wait_budget_ns();
@@ -399,10 +442,15 @@ mala_status mala_bwd(const void* Q, const void* K, const void* V, const void* O,
   if (dtype == MALA_BF16 && d != 64 && d != 128) return MALA_ERR_UNSUPPORTED;
   if (dtype == MALA_FP32 && d > 128) return MALA_ERR_UNSUPPORTED;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t T = (static_cast<size_t>(L) + kTile - 1) / kTile;
+  bool margin_ok = true;
+  float* margin = debug_margin(static_cast<size_t>(B) * H * T * T, margin_ok);
+  if (!margin_ok) return MALA_ERR_INVALID_ARG;
   const size_t need = bwd_workspace_bytes(B, H, H_kv, L, d, dtype);
   return with_workspace(workspace, workspace_bytes, need, st, [&](uint8_t* ws) -> mala_status {
+    if (!debug_margin_clear(margin, static_cast<size_t>(B) * H * T * T, st)) return MALA_ERR_CUDA;
     return bwd_dispatch(Q, K, V, O, LSE, dO, dQ, dK, dV, B, H, H_kv, L, d, dtype, scale, tau,
-                        flags, ws, tile_mask, wait_budget_ns(), st);
+                        flags, ws, tile_mask, margin, wait_budget_ns(), st);
   });
 }
 
@@ -435,10 +483,14 @@ mala_status mala_decode(const void* q, const void* Kc, const void* Vc, void* O, 
   if (dtype == MALA_BF16 && H / H_kv > 8) return MALA_ERR_UNSUPPORTED;  // up to 8 per group
   if (dtype == MALA_FP32 && d > 128) return MALA_ERR_UNSUPPORTED;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  bool margin_ok = true;
+  float* margin = debug_margin(static_cast<size_t>(B) * H * T, margin_ok);
+  if (!margin_ok) return MALA_ERR_INVALID_ARG;
   const size_t need = decode_workspace_bytes(B, H, H_kv, Nk, d, dtype, num_splits);
   return with_workspace(workspace, workspace_bytes, need, st, [&](uint8_t* ws) -> mala_status {
+    if (!debug_margin_clear(margin, static_cast<size_t>(B) * H * T, st)) return MALA_ERR_CUDA;
     return decode_dispatch(q, Kc, Vc, O, LSE, B, H, H_kv, Nk, d, dtype, scale, tau, num_splits,
-                           flags, ws, tile_mask, wait_budget_ns(), st);
+                           flags, ws, tile_mask, margin, wait_budget_ns(), st);
   });
 }
 

@@ -77,6 +77,7 @@ struct BwdParams {
   __nv_bfloat16* dK;     // [B, L, Hkv, D]
   __nv_bfloat16* dV;
   uint8_t* tile_mask;    // [B, H, T, T] or null
+  float* tile_margin;    // [B, H, T, T] debug margins (natural log) or null
   unsigned long long* stats;  // call statistics (kStatsOffset) or null
   uint32_t* err;
   uint32_t* sched;
@@ -471,6 +472,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
               }
           }
           keep = named_bar_or(1, 256, ymax >= 0.f);
+          if (p.tile_margin) {
+            // debug: the tile's margin max over legal entries of log P - log(tau / L_q),
+            // natural-log units
+            const float x = warp_max_f32(ymax);
+            if (lane == 0)
+              atomic_max_f32(p.tile_margin + ((static_cast<size_t>(w.b) * p.H + h) * p.T + i) * p.T +
+                                 w.j,
+                             x * kLn2);
+          }
         } else {
           named_bar_sync(1, 256);  // every S^T load done before P overwrites it
         }
@@ -717,7 +727,7 @@ size_t bwd_workspace_bytes(int B, int H, int Hkv, int L, int d, int dtype) {
 mala_status fp32_bwd(const float* Q, const float* K, const float* V, const float* O,
                      const float* LSE, const float* dO, float* dQ, float* dK, float* dV, int B,
                      int H, int Hkv, int L, int d, float scale, float tau, bool screen,
-                     uint8_t* ws, uint8_t* tile_mask, cudaStream_t stream);
+                     uint8_t* ws, uint8_t* tile_mask, float* tile_margin, cudaStream_t stream);
 
 template <int D, bool kScreen>
 static cudaError_t launch_bwd_main(const CUtensorMap& tq, const CUtensorMap& tk,
@@ -759,8 +769,8 @@ static bool make_f32_reduce_map(CUtensorMap* m, void* base, int n0, int n1, int 
 mala_status bwd_dispatch(const void* Q, const void* K, const void* V, const void* O,
                          const float* LSE, const void* dO, void* dQ, void* dK, void* dV, int B,
                          int H, int Hkv, int L, int d, int dtype, float scale, float tau,
-                         unsigned flags, uint8_t* ws, uint8_t* tile_mask, uint64_t budget_ns,
-                         cudaStream_t stream) {
+                         unsigned flags, uint8_t* ws, uint8_t* tile_mask, float* tile_margin,
+                         uint64_t budget_ns, cudaStream_t stream) {
   const bool screen = (tau > 0.f) || (flags & MALA_FLAG_ALWAYS_TEST);
   if (cudaMemsetAsync(ws + kStatsOffset, 0, 3 * sizeof(unsigned long long), stream) !=
       cudaSuccess)
@@ -770,7 +780,7 @@ mala_status bwd_dispatch(const void* Q, const void* K, const void* V, const void
                     static_cast<const float*>(V), static_cast<const float*>(O), LSE,
                     static_cast<const float*>(dO), static_cast<float*>(dQ),
                     static_cast<float*>(dK), static_cast<float*>(dV), B, H, Hkv, L, d, scale,
-                    tau, screen, ws, tile_mask, stream);
+                    tau, screen, ws, tile_mask, tile_margin, stream);
   const int T = (L + kTile - 1) / kTile;
   CUtensorMap tq, tk, tv, tdo;
   if (!make_tile_map(&tq, Q, d, H, L, B) || !make_tile_map(&tk, K, d, Hkv, L, B) ||
@@ -805,6 +815,7 @@ mala_status bwd_dispatch(const void* Q, const void* K, const void* V, const void
   p.dK = static_cast<__nv_bfloat16*>(dK);
   p.dV = static_cast<__nv_bfloat16*>(dV);
   p.tile_mask = tile_mask;
+  p.tile_margin = tile_margin;
   p.stats = reinterpret_cast<unsigned long long*>(ws + kStatsOffset);
   p.err = hdr + kHdrError;
   p.sched = hdr + kHdrSched0;

@@ -31,6 +31,26 @@ __device__ __forceinline__ void stats_add(unsigned long long* stats, uint32_t le
   if (retained) atomicAdd(stats + 1, static_cast<unsigned long long>(retained));
   if (v_loaded) atomicAdd(stats + 2, static_cast<unsigned long long>(v_loaded));
 }
+
+// Debug margins: float max into a global buffer whose entries start as the all-ones bit
+// pattern (written by the host before the launch).  Non-negative values are combined as
+// signed integers and negative ones as unsigned integers, which both order IEEE floats
+// correctly; the all-ones start value is below every float under both views, so the
+// first arrival always wins.  -0 is folded into +0 first.
+__device__ __forceinline__ void atomic_max_f32(float* addr, float v) {
+  if (v == 0.f) v = 0.f;
+  if (v >= 0.f)
+    atomicMax(reinterpret_cast<int*>(addr), __float_as_int(v));
+  else
+    atomicMin(reinterpret_cast<unsigned int*>(addr), __float_as_uint(v));
+}
+
+// Warp-wide maximum (all 32 lanes must call).
+__device__ __forceinline__ float warp_max_f32(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
 #endif
 
 // One query block of one sequence of a packed (varlen) batch, in the order the
@@ -53,6 +73,7 @@ struct FwdParams {
   void* O;            // [B, L, H, D] bf16
   float* LSE;         // [B, H, L]
   uint8_t* tile_mask; // [B, H, T, Tk] or null
+  float* tile_margin; // [B, H, T, Tk] debug margins (natural log) or null
   uint32_t* err;      // device error word
   uint32_t* sched;    // persistent scheduler counter (zeroed before launch)
   uint64_t budget_ns;

@@ -78,6 +78,7 @@ struct DecParams {
   float* part_z;           // [B, H, S] (natural log)
   uint32_t* tickets;       // [B * Hkv]
   uint8_t* tile_mask;      // [B, H, T] or null
+  float* tile_margin;      // [B, H, T] debug margins (natural log) or null
   unsigned long long* stats;  // call statistics (kStatsOffset) or null
   uint32_t* err;
   uint64_t budget_ns;
@@ -389,8 +390,8 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, 1)
             tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 2));
             tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 4));
             bool k = hd < G;
-            if (kScreen && k)
-              k = (l_h[hs] == 0.f) || (tmax >= m_h[hs] + __log2f(l_h[hs]) + p.thr2);
+            const float cut = m_h[hs] + __log2f(l_h[hs]) + p.thr2;
+            if (kScreen && k) k = (l_h[hs] == 0.f) || (tmax >= cut);
             const uint32_t bal = __ballot_sync(0xffffffffu, k);
             keep |= ((bal & 1u) | ((bal >> 7) & 2u) | ((bal >> 14) & 4u) | ((bal >> 21) & 8u))
                     << (4 * hs);
@@ -409,6 +410,11 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, 1)
               if (dw == 0) sh.alpha[slot][hd] = k ? alpha_prev[hs] : 1.f;
               if (p.tile_mask && dw == 0 && hd < G)
                 p.tile_mask[(static_cast<size_t>(b) * p.H + g * G + hd) * p.T + t] = k ? 1 : 0;
+              // debug: the margin of the test in natural-log units (+inf on a split's
+              // first tile)
+              if (kScreen && p.tile_margin && dw == 0 && hd < G)
+                p.tile_margin[(static_cast<size_t>(b) * p.H + g * G + hd) * p.T + t] =
+                    (l_h[hs] == 0.f) ? INFINITY : (tmax - cut) * kLn2;
             }
           }
           const uint32_t bal = keep;  // nonzero: some head keeps the tile (warp-uniform)
@@ -606,7 +612,8 @@ size_t decode_workspace_bytes(int B, int H, int Hkv, int Nk, int d, int dtype, i
 
 mala_status fp32_decode(const float* q, const float* K, const float* V, float* O, float* LSE,
                         int B, int H, int Hkv, int Nk, int d, float scale, float tau, int S,
-                        bool screen, uint8_t* ws, uint8_t* tile_mask, cudaStream_t stream);
+                        bool screen, uint8_t* ws, uint8_t* tile_mask, float* tile_margin,
+                        cudaStream_t stream);
 
 template <int D, bool kScreen, int HS>
 static cudaError_t launch_decode(const CUtensorMap& tk, const CUtensorMap& tv,
@@ -622,7 +629,8 @@ static cudaError_t launch_decode(const CUtensorMap& tk, const CUtensorMap& tv,
 mala_status decode_dispatch(const void* q, const void* K, const void* V, void* O, float* LSE,
                             int B, int H, int Hkv, int Nk, int d, int dtype, float scale,
                             float tau, int num_splits, unsigned flags, uint8_t* ws,
-                            uint8_t* tile_mask, uint64_t budget_ns, cudaStream_t stream) {
+                            uint8_t* tile_mask, float* tile_margin, uint64_t budget_ns,
+                            cudaStream_t stream) {
   const bool screen = (tau > 0.f) || (flags & MALA_FLAG_ALWAYS_TEST);
   if (cudaMemsetAsync(ws + kStatsOffset, 0, 3 * sizeof(unsigned long long), stream) !=
       cudaSuccess)
@@ -630,7 +638,7 @@ mala_status decode_dispatch(const void* q, const void* K, const void* V, void* O
   if (dtype == MALA_FP32)
     return fp32_decode(static_cast<const float*>(q), static_cast<const float*>(K),
                        static_cast<const float*>(V), static_cast<float*>(O), LSE, B, H, Hkv, Nk,
-                       d, scale, tau, num_splits, screen, ws, tile_mask, stream);
+                       d, scale, tau, num_splits, screen, ws, tile_mask, tile_margin, stream);
   if (H / Hkv > 8) return MALA_ERR_UNSUPPORTED;  // the kernel packs up to 8 heads per group
   CUtensorMap tk, tv;
   if (!make_tile_map(&tk, K, d, Hkv, Nk, B) || !make_tile_map(&tv, V, d, Hkv, Nk, B))
@@ -650,6 +658,7 @@ mala_status decode_dispatch(const void* q, const void* K, const void* V, void* O
   p.part_z = p.part_o + static_cast<size_t>(B) * H * num_splits * d;
   p.tickets = reinterpret_cast<uint32_t*>(part + ((part_bytes + 255) / 256) * 256);
   p.tile_mask = tile_mask;
+  p.tile_margin = tile_margin;
   p.stats = reinterpret_cast<unsigned long long*>(ws + kStatsOffset);
   p.err = reinterpret_cast<uint32_t*>(ws) + kHdrError;
   p.budget_ns = budget_ns;

@@ -13,6 +13,7 @@
 // cleared on the stream at the start of every call; two calls whose work overlaps on
 // the GPU (for example on two streams at once) race on it and must be serialised.
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -26,7 +27,8 @@ namespace mala {
 mala_status decode_dispatch(const void* q, const void* K, const void* V, void* O, float* LSE,
                             int B, int H, int Hkv, int Nk, int d, int dtype, float scale,
                             float tau, int num_splits, unsigned flags, uint8_t* ws,
-                            uint8_t* tile_mask, uint64_t budget_ns, cudaStream_t stream);
+                            uint8_t* tile_mask, float* tile_margin, uint64_t budget_ns,
+                            cudaStream_t stream);
 size_t decode_workspace_bytes(int B, int H, int Hkv, int Nk, int d, int dtype, int num_splits);
 int decode_auto_splits(int B, int Hkv, int Nk);
 bool common_args_ok(int B, int H, int Hkv, int L, int d, int dtype, float scale, float tau);
@@ -42,17 +44,43 @@ static __device__ __align__(256) uint8_t g_noalloc_scratch[MALA_DECODE_NOALLOC_S
 constexpr int kMaxDevices = 64;
 std::mutex g_setup_mutex;
 void* g_scratch_ptr[kMaxDevices] = {};
+void* g_scratch_ctx[kMaxDevices] = {};  // context the cached address belongs to
 
-// Device address of the scratch on the current device (looked up once per device).
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+
+// The current driver context (null if it cannot be queried).
+void* current_context() {
+  static CtxGetCurrentFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(f);
+  });
+  CUcontext ctx = nullptr;
+  if (!fn || fn(&ctx) != CUDA_SUCCESS) return nullptr;
+  return ctx;
+}
+
+// Device address of the scratch on the current device.  It is looked up once per device
+// and context: after the primary context of a device has been destroyed and recreated
+// (cudaDeviceReset) the module is loaded again, possibly elsewhere, so a cached address
+// from the old context is looked up afresh.
 mala_status scratch_for_current_device(uint8_t** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MALA_ERR_CUDA;
+  // (before the runtime's first call on this thread no context may be current yet: the
+  // lookup below then runs, and it makes the device's primary context current)
+  void* ctx = current_context();
   std::lock_guard<std::mutex> lock(g_setup_mutex);
-  if (!g_scratch_ptr[dev]) {
+  if (!g_scratch_ptr[dev] || !ctx || g_scratch_ctx[dev] != ctx) {
     void* ptr = nullptr;
     if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr)
       return MALA_ERR_CUDA;
     g_scratch_ptr[dev] = ptr;
+    g_scratch_ctx[dev] = current_context();
   }
   *out = static_cast<uint8_t*>(g_scratch_ptr[dev]);
   return MALA_OK;
@@ -87,5 +115,5 @@ extern "C" mala_status mala_decode_noalloc(const void* q, const void* Kc, const 
   // the error word and counters must start at zero; the launcher clears the tickets
   if (cudaMemsetAsync(ws, 0, kWorkspaceHeader, s) != cudaSuccess) return MALA_ERR_CUDA;
   return decode_dispatch(q, Kc, Vc, O, LSE, B, H, H_kv, Nk, d, dtype, scale, tau, num_splits,
-                         flags, ws, tile_mask, wait_budget_ns(), s);
+                         flags, ws, tile_mask, nullptr, wait_budget_ns(), s);
 }

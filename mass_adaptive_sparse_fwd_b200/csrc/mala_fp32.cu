@@ -41,7 +41,8 @@ __global__ void __launch_bounds__(kF32Threads)
     fp32_fwd_kernel(const float* __restrict__ Q, const float* __restrict__ K,
                     const float* __restrict__ V, float* __restrict__ O, float* __restrict__ LSE,
                     int B, int H, int Hkv, int L, int Lk, int d, float scale, float tau,
-                    bool screen, uint8_t* tile_mask, unsigned long long* stats) {
+                    bool screen, uint8_t* tile_mask, float* tile_margin,
+                    unsigned long long* stats) {
   extern __shared__ float fsm[];
   float* sK = fsm;             // [128][d]
   float* sV = fsm + kTile * d;  // [128][d]
@@ -82,7 +83,11 @@ __global__ void __launch_bounds__(kF32Threads)
       if (legal) { has = true; rmax = fmaxf(rmax, s[kk]); }
     }
     bool mine = has;
-    if (screen && has && l > 0.f) mine = (rmax - m - logf(l) - theta) >= 0.f;
+    const float x = (l > 0.f) ? rmax - m - logf(l) - theta : INFINITY;
+    if (screen && has && l > 0.f) mine = x >= 0.f;
+    // debug: the tile's margin, max over rows with a legal key (natural-log units)
+    if (screen && has && tile_margin)
+      atomic_max_f32(tile_margin + ((static_cast<size_t>(b) * H + h) * T + i) * Tk + j, x);
     const bool keep = __syncthreads_or(mine) != 0;
     if (r == 0) {
       stats_add(stats, 1, keep ? 1 : 0, 0);
@@ -127,7 +132,7 @@ __global__ void __launch_bounds__(kF32Threads)
                        const float* __restrict__ dO, const float* __restrict__ Dsum,
                        float* __restrict__ dK, float* __restrict__ dV, int B, int H, int Hkv,
                        int L, int d, float scale, float tau, bool screen, uint8_t* tile_mask,
-                       unsigned long long* stats) {
+                       float* tile_margin, unsigned long long* stats) {
   extern __shared__ float fsm[];
   float* sQ = fsm;               // [128][d]
   float* sdO = fsm + kTile * d;  // [128][d]
@@ -167,12 +172,17 @@ __global__ void __launch_bounds__(kF32Threads)
       }
       __syncthreads();
       bool mine = false;
+      float ymax = -INFINITY;  // this key's largest log P - log(tau / L_q) in the tile
       for (int qq = 0; qq < kTile; ++qq) {
         const int q = i * kTile + qq;
         if (!kvalid || q >= L || q < k) continue;
         const float s = scale * dot_rows(sQ + qq * d, kv, d);
-        if (!screen || s - sL[qq] - sT[qq] >= 0.f) mine = true;
+        const float y = s - sL[qq] - sT[qq];
+        ymax = fmaxf(ymax, y);
+        if (!screen || y >= 0.f) mine = true;
       }
+      if (screen && tile_margin && ymax != -INFINITY)
+        atomic_max_f32(tile_margin + ((static_cast<size_t>(b) * H + h) * T + i) * T + j, ymax);
       const bool keep = __syncthreads_or(mine) != 0;
       if (r == 0) {
         stats_add(stats, 1, keep ? 1 : 0, 0);
@@ -268,7 +278,7 @@ __global__ void __launch_bounds__(kF32Threads)
                              const float* __restrict__ V, float* __restrict__ part_o,
                              float* __restrict__ part_z, int B, int H, int Hkv, int Nk, int d,
                              int S, float scale, float tau, bool screen, uint8_t* tile_mask,
-                             unsigned long long* stats) {
+                             float* tile_margin, unsigned long long* stats) {
   __shared__ float sq[128], sp[kTile], red[kTile];
   const int T = (Nk + kTile - 1) / kTile;
   const int s = blockIdx.x % S;
@@ -296,7 +306,10 @@ __global__ void __launch_bounds__(kF32Threads)
     const float rmax = red[0];
     __syncthreads();
     bool keep = true;
-    if (screen && l > 0.f) keep = (rmax - m - logf(l) - theta) >= 0.f;
+    const float x = (l > 0.f) ? rmax - m - logf(l) - theta : INFINITY;
+    if (screen && l > 0.f) keep = x >= 0.f;
+    if (r == 0 && screen && tile_margin)
+      tile_margin[(static_cast<size_t>(b) * H + h) * T + t] = x;  // debug margin
     if (r == 0) {
       // this path loads V per head: one V tile per retained (head, tile)
       stats_add(stats, 1, keep ? 1 : 0, keep ? 1 : 0);
@@ -357,7 +370,7 @@ cudaError_t set_smem(const void* fn, int bytes) {
 
 mala_status fp32_fwd(const float* Q, const float* K, const float* V, float* O, float* LSE, int B,
                      int H, int Hkv, int L, int Lk, int d, float scale, float tau, bool screen,
-                     uint8_t* ws, uint8_t* tile_mask, cudaStream_t stream) {
+                     uint8_t* ws, uint8_t* tile_mask, float* tile_margin, cudaStream_t stream) {
   const int T = (L + kTile - 1) / kTile;
   const int smem = 2 * kTile * d * static_cast<int>(sizeof(float));
   unsigned long long* stats =
@@ -365,14 +378,14 @@ mala_status fp32_fwd(const float* Q, const float* K, const float* V, float* O, f
   if (set_smem(reinterpret_cast<const void*>(fp32_fwd_kernel), smem) != cudaSuccess)
     return MALA_ERR_CUDA;
   fp32_fwd_kernel<<<B * H * T, kF32Threads, smem, stream>>>(
-      Q, K, V, O, LSE, B, H, Hkv, L, Lk, d, scale, tau, screen, tile_mask, stats);
+      Q, K, V, O, LSE, B, H, Hkv, L, Lk, d, scale, tau, screen, tile_mask, tile_margin, stats);
   return cudaGetLastError() == cudaSuccess ? MALA_OK : MALA_ERR_CUDA;
 }
 
 mala_status fp32_bwd(const float* Q, const float* K, const float* V, const float* O,
                      const float* LSE, const float* dO, float* dQ, float* dK, float* dV, int B,
                      int H, int Hkv, int L, int d, float scale, float tau, bool screen,
-                     uint8_t* ws, uint8_t* tile_mask, cudaStream_t stream) {
+                     uint8_t* ws, uint8_t* tile_mask, float* tile_margin, cudaStream_t stream) {
   const int T = (L + kTile - 1) / kTile;
   float* Dsum = reinterpret_cast<float*>(ws + kWorkspaceHeader);
   const long long rows = static_cast<long long>(B) * L * H;
@@ -384,7 +397,7 @@ mala_status fp32_bwd(const float* Q, const float* K, const float* V, const float
       set_smem(reinterpret_cast<const void*>(fp32_bwd_q_kernel), smem_q) != cudaSuccess)
     return MALA_ERR_CUDA;
   fp32_bwd_kv_kernel<<<B * Hkv * T, kF32Threads, smem_kv, stream>>>(
-      Q, K, V, LSE, dO, Dsum, dK, dV, B, H, Hkv, L, d, scale, tau, screen, tile_mask,
+      Q, K, V, LSE, dO, Dsum, dK, dV, B, H, Hkv, L, d, scale, tau, screen, tile_mask, tile_margin,
       reinterpret_cast<unsigned long long*>(ws + kStatsOffset));
   fp32_bwd_q_kernel<<<B * H * T, kF32Threads, smem_q, stream>>>(Q, K, V, LSE, dO, Dsum, dQ, B, H,
                                                                 Hkv, L, d, scale, tau, screen);
@@ -393,11 +406,12 @@ mala_status fp32_bwd(const float* Q, const float* K, const float* V, const float
 
 mala_status fp32_decode(const float* q, const float* K, const float* V, float* O, float* LSE,
                         int B, int H, int Hkv, int Nk, int d, float scale, float tau, int S,
-                        bool screen, uint8_t* ws, uint8_t* tile_mask, cudaStream_t stream) {
+                        bool screen, uint8_t* ws, uint8_t* tile_mask, float* tile_margin,
+                        cudaStream_t stream) {
   float* part_o = reinterpret_cast<float*>(ws + kWorkspaceHeader);
   float* part_z = part_o + static_cast<size_t>(B) * H * S * d;
   fp32_decode_split_kernel<<<B * H * S, kF32Threads, 0, stream>>>(
-      q, K, V, part_o, part_z, B, H, Hkv, Nk, d, S, scale, tau, screen, tile_mask,
+      q, K, V, part_o, part_z, B, H, Hkv, Nk, d, S, scale, tau, screen, tile_mask, tile_margin,
       reinterpret_cast<unsigned long long*>(ws + kStatsOffset));
   fp32_decode_merge_kernel<<<B * H, 128, 0, stream>>>(part_o, part_z, O, LSE, B * H, S, d);
   return cudaGetLastError() == cudaSuccess ? MALA_OK : MALA_ERR_CUDA;

@@ -404,8 +404,19 @@ __global__ void __launch_bounds__(384, 1)
         const float rmax = rraw * p.scale_log2;
         bool keep = true;
         if (kScreen) {
-          const bool mine = (rmax != NEG_INF) && (l == 0.f || rmax >= m2 + __log2f(l) + thr2);
+          const float cut = m2 + __log2f(l) + thr2;
+          const bool mine = (rmax != NEG_INF) && (l == 0.f || rmax >= cut);
           keep = named_bar_or(1 + s, 128, mine);
+          if (p.tile_margin) {
+            // debug: the tile's margin max_q (rowmax - cut) in natural-log units (+inf for
+            // a row's first retained tile, -inf for rows without a legal key)
+            float x = (rmax == NEG_INF) ? NEG_INF : (l == 0.f ? INFINITY : rmax - cut);
+            x = warp_max_f32(x);
+            if (lane == 0)
+              atomic_max_f32(p.tile_margin + ((static_cast<size_t>(w.b) * p.H + h) * p.T + w.i) *
+                                                 p.Tk + j,
+                             x * kLn2);
+          }
           if (*ast.flag) { ok = false; break; }
         }
         if (p.tile_mask && r == 0)

@@ -29,13 +29,17 @@ EXPORTED = ("mala_fwd", "mala_fwd_prefill", "mala_fwd_varlen", "mala_bwd", "mala
             "mala_selftest_wait_timeout",
             "mala_fwd_workspace_bytes",
             "mala_bwd_workspace_bytes", "mala_decode_workspace_bytes", "mala_decode_num_splits",
-            "mala_read_device_error", "mala_set_wait_budget_ns", "mala_status_string",
-            "mala_version")
+            "mala_read_device_error", "mala_set_wait_budget_ns", "mala_set_debug",
+            "mala_status_string", "mala_version")
 
 
 class MalaStats(ctypes.Structure):
     _fields_ = [("legal_tiles", ctypes.c_uint64), ("retained_tiles", ctypes.c_uint64),
                 ("v_tiles_loaded", ctypes.c_uint64)]
+
+
+class MalaDebug(ctypes.Structure):
+    _fields_ = [("tile_margin", ctypes.c_void_p), ("tile_margin_count", ctypes.c_size_t)]
 
 
 class MalaError(RuntimeError):
@@ -84,6 +88,8 @@ def load_library(path: str = _LIB_PATH) -> ctypes.CDLL:
     lib.mala_selftest_wait_timeout.restype = ci
     lib.mala_get_stats.argtypes = [vp, vp, ctypes.POINTER(MalaStats)]
     lib.mala_get_stats.restype = ci
+    lib.mala_set_debug.argtypes = [ctypes.POINTER(MalaDebug)]
+    lib.mala_set_debug.restype = ci
     lib.mala_status_string.argtypes = [ci]
     lib.mala_status_string.restype = ctypes.c_char_p
     lib.mala_version.restype = ci
@@ -408,3 +414,34 @@ def selftest_wait_timeout(workspace: torch.Tensor, budget_ns: int, stream=None):
 
 def set_wait_budget_ns(ns: int):
     _check("mala_set_wait_budget_ns", _lib.mala_set_wait_budget_ns(int(ns)))
+
+
+def set_debug(tile_margin=None):
+    """Registers (or, with None, clears) a float32 CUDA buffer that receives the margin of
+    every retention test of this thread's later forward, prefill, backward and decode
+    calls, in the layout of their tile masks (see ``mala_set_debug`` in the header)."""
+    if tile_margin is None:
+        _check("mala_set_debug", _lib.mala_set_debug(None))
+        return
+    if not isinstance(tile_margin, torch.Tensor) or tile_margin.dtype != torch.float32 or \
+            not tile_margin.is_contiguous():
+        raise TypeError("set_debug: tile_margin must be a contiguous float32 tensor")
+    _need_cuda("set_debug", tile_margin.device)
+    dbg = MalaDebug(tile_margin.data_ptr(), tile_margin.numel())
+    _check("mala_set_debug", _lib.mala_set_debug(ctypes.byref(dbg)))
+
+
+class debug_margins:
+    """Context manager: ``with debug_margins(buf): mala_fwd(...)`` fills ``buf`` with the
+    call's tile margins and turns the hook off on exit."""
+
+    def __init__(self, tile_margin):
+        self.buf = tile_margin
+
+    def __enter__(self):
+        set_debug(self.buf)
+        return self.buf
+
+    def __exit__(self, *exc):
+        set_debug(None)
+        return False

@@ -131,9 +131,13 @@ def evaluate(Q, K, V, scale, mala_mask, tile=TILE, device="cpu"):
     return out
 
 
-def run_study(workload="prevvar8k", seeds=(8, 18, 28, 38), tau=1.0, L=None, device="cuda"):
+def run_study(workload="prevvar8k", seeds=(8, 18, 28, 38), tau=1.0, L=None, device="cuda",
+              on_decisions=None):
     """MALA's decisions from the GPU forward (tile mask) on X seeded instances of a
-    workload (optionally at another length L), then ``evaluate``."""
+    workload (optionally at another length L), then ``evaluate``.  ``on_decisions``, if
+    given, is called as on_decisions(w, inp, mask, margin) for every instance with the
+    exact mask the study consumes and the forward's exported test margins (the
+    library's debug hook is on for those calls), so a caller can audit the decisions."""
     import torch
 
     from . import mala, synth
@@ -148,8 +152,15 @@ def run_study(workload="prevvar8k", seeds=(8, 18, 28, 38), tau=1.0, L=None, devi
                    for n in ("Q", "K", "V"))
         T = mala.n_tiles(inp["Q"].shape[1])
         m = torch.zeros((w.B, w.H, T, T), dtype=torch.uint8, device=device)
-        mala.mala_fwd(q, k, v, w.scale, tau, tile_mask=m)
+        if on_decisions is None:
+            mala.mala_fwd(q, k, v, w.scale, tau, tile_mask=m)
+        else:
+            margin = torch.empty(w.B * w.H * T * T, dtype=torch.float32, device=device)
+            with mala.debug_margins(margin):
+                mala.mala_fwd(q, k, v, w.scale, tau, tile_mask=m)
         torch.cuda.synchronize()
+        if on_decisions is not None:
+            on_decisions(w, inp, m.cpu().numpy(), margin.view(w.B, w.H, T, T).cpu().numpy())
         Qs.append(inp["Q"][:1]); Ks.append(inp["K"][:1]); Vs.append(inp["V"][:1])
         masks.append(m.cpu().numpy()[:1])
     res = evaluate(np.concatenate(Qs), np.concatenate(Ks), np.concatenate(Vs), base.scale,

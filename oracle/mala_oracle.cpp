@@ -13,7 +13,7 @@
 //   §2.3  the same forward serves inference prefill: orc_mala_prefill takes a chunk of
 //         queries at the end of a longer key sequence (causal offset Nk - Nq)
 //
-// Conventions (each one a reading of the page, listed in the design doc):
+// Conventions (each one a reading of the page where it is silent or ambiguous):
 //   * scores s = scale * <q, k>, natural exp / log (§2.1 absorbs the scale into Q)
 //   * square tiles of `blk` rows/keys; tile (i, j) = query block i, key block j
 //   * forward visits j = i, i-1, ..., 0 (diagonal first, A.1); only legal tiles

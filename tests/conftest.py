@@ -19,3 +19,21 @@ def orc():
 
     oracle.build()
     return oracle
+
+
+def pytest_terminal_summary(terminalreporter):
+    # decision-parity and output figures recorded by the GPU parity tests
+    parity = sys.modules.get("tests.parity")
+    if parity is not None and parity.REPORT:
+        terminalreporter.write_line("")
+        for line in parity.format_report(parity.REPORT).splitlines():
+            terminalreporter.write_line(line)
+        try:
+            import json
+
+            out = os.path.join(ROOT, "gpurun_out")
+            if os.path.isdir(out):
+                with open(os.path.join(out, "parity_report.json"), "w") as f:
+                    json.dump(parity.REPORT, f, indent=1)
+        except OSError:
+            pass

@@ -19,13 +19,19 @@ def mala():
     return m
 
 
-def run_fwd(mala, inp, w, tau, flags=0):
+def run_fwd(mala, inp, w, tau, flags=0, debug=True):
     Q, K, V = (P.to_dev(inp[k], w.dtype) for k in ("Q", "K", "V"))
     B, L, H, d = Q.shape
     T = mala.n_tiles(L)
     mask = torch.full((B, H, T, T), 255, dtype=torch.uint8, device="cuda")
+    margin = P.margin_buffer(B * H * T * T)
     ws = mala.alloc_workspace(mala.fwd_workspace_bytes(B, H, K.shape[2], L, d), "cuda")
-    O, LSE = mala.mala_fwd(Q, K, V, w.scale, tau, flags=flags, workspace=ws, tile_mask=mask)
+    if debug:
+        with mala.debug_margins(margin):
+            O, LSE = mala.mala_fwd(Q, K, V, w.scale, tau, flags=flags, workspace=ws,
+                                   tile_mask=mask)
+    else:
+        O, LSE = mala.mala_fwd(Q, K, V, w.scale, tau, flags=flags, workspace=ws, tile_mask=mask)
     torch.cuda.synchronize()
     assert mala.read_device_error(ws) == 0
     mask = mask.cpu().numpy()
@@ -33,11 +39,19 @@ def run_fwd(mala, inp, w, tau, flags=0):
     legal = P.fwd_legal(B, H, T)
     st = mala.get_stats(ws)
     assert st["legal_tiles"] == legal.sum() and st["retained_tiles"] == (mask[legal] == 1).sum()
-    return O.float().cpu().numpy(), LSE.cpu().numpy(), mask
+    return (O.float().cpu().numpy(), LSE.cpu().numpy(), mask,
+            margin.view(B, H, T, T).cpu().numpy())
 
 
-def check_fwd(orc, mala, w, inp, tau, units=None, flags=0):
-    O, LSE, mask = run_fwd(mala, inp, w, tau, flags)
+def label_of(kind, w, inp, tau, flags=0):
+    B, L, H, d = inp["Q"].shape
+    return (f"{kind} {w.name}:{w.structure} B{B} H{H}/{inp['K'].shape[2]} L{L} d{d} "
+            f"{w.dtype} tau={tau:g}"
+            + (" always-test" if flags else ""))
+
+
+def check_fwd(orc, mala, w, inp, tau, units=None, flags=0, max_flips=0):
+    O, LSE, mask, gmargin = run_fwd(mala, inp, w, tau, flags)
     B, L, H, d = inp["Q"].shape
     T = (L + 127) // 128
     legal_all = P.fwd_legal(B, H, T)
@@ -48,16 +62,19 @@ def check_fwd(orc, mala, w, inp, tau, units=None, flags=0):
     oO, oLSE, omask, omargin = orc.mala_fwd(inp["Q"], inp["K"], inp["V"], w.scale, tau,
                                             units=units, force=force)
     legal = P.fwd_legal(B, H, T, units)
-    band = P.tile_bands(inp["Q"], inp["K"], w.scale, H // inp["K"].shape[2])
-    n, near, bad, worst = P.compare_masks(mask, omargin, band, legal)
-    assert bad == 0, f"{bad} tile decisions differ beyond the band (worst margin {worst})"
+    label = label_of("fwd", w, inp, tau, flags)
+    row = {"flips": 0}
+    if tau > 0 or flags:
+        row = P.compare_decisions(label, "fp32" if w.dtype == "fp32" else "fwd", mask, gmargin,
+                                  omargin, legal, max_flips)
     rows = np.isfinite(oLSE)  # [B,H,L] rows the oracle computed
     rows_o = np.transpose(rows, (0, 2, 1))  # [B,L,H]
-    P.check_output(O, oO, rows_o)
+    P.check_output(O, oO, rows_o, label)
     assert np.abs(LSE - oLSE)[rows].max() < P.LSE_ABS
     if tau == 0:
         assert (mask[legal_all] == 1).all()
-    return {"tiles": n, "near": near, "retained": float(mask[legal_all].mean())}
+    return {"tiles": int(legal.sum()), "flips": row["flips"],
+            "retained": float(mask[legal_all].mean()), "margin": gmargin}
 
 
 @pytest.mark.parametrize("tau", [0.0, 1.0])
@@ -142,3 +159,13 @@ def test_fwd_prevtok32k_sampled(orc, mala):
     T = w.L // 128
     st = check_fwd(orc, mala, w, inp, 1.0, units=_units(w.B, w.H, T, 6, seed=9))
     assert st["retained"] < 0.05
+
+
+def test_fwd_debug_hook_changes_nothing(orc, mala):
+    """The margin export does not alter the forward: same decisions, bitwise equal O and
+    LSE with the hook on and off."""
+    w, inp = synth.small_training(B=1, H=4, Hkv=1, L=2048, d=128, structure="prev_token", seed=4)
+    a = run_fwd(mala, inp, w, 1.0, debug=True)
+    b = run_fwd(mala, inp, w, 1.0, debug=False)
+    assert np.array_equal(a[2], b[2])
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])

@@ -43,31 +43,17 @@ def prefill_legal(B, H, Nq, Nk, units=None):
     return out
 
 
-def prefill_bands(Qc, K, scale, G):
-    """Decision band per tile [B,H,Tq,Tk]: fp32 score rounding of the tile's largest
-    |q| |k| product (as for the square forward) plus the log2 / running-sum slack."""
-    B, Nq, H, d = Qc.shape
-    Nk = K.shape[1]
-    Tq, Tk = -(-Nq // 128), -(-Nk // 128)
-    qn = np.linalg.norm(Qc.astype(np.float64), axis=-1)
-    kn = np.linalg.norm(K.astype(np.float64), axis=-1)
-    qn = np.pad(qn, ((0, 0), (0, Tq * 128 - Nq), (0, 0))).reshape(B, Tq, 128, H).max(axis=2)
-    kn = np.pad(kn, ((0, 0), (0, Tk * 128 - Nk), (0, 0))).reshape(B, Tk, 128, -1).max(axis=2)
-    kn = np.repeat(kn, G, axis=2)
-    err = d * 2.0 ** -22 * scale * qn.transpose(0, 2, 1)[:, :, :, None] * \
-        kn.transpose(0, 2, 1)[:, :, None, :]
-    return 1e-6 + 1e-5 + err
-
-
 def run_prefill(mala, Qc, K, V, w, tau, flags=0):
     Q, Kd, Vd = (P.to_dev(x, w.dtype) for x in (Qc, K, V))
     B, Nq, H, d = Q.shape
     Nk, Hkv = Kd.shape[1], Kd.shape[2]
     Tq, Tk = mala.n_tiles(Nq), mala.n_tiles(Nk)
     mask = torch.full((B, H, Tq, Tk), 255, dtype=torch.uint8, device="cuda")
+    margin = P.margin_buffer(B * H * Tq * Tk)
     ws = mala.alloc_workspace(mala.fwd_workspace_bytes(B, H, Hkv, Nq, d), "cuda")
-    O, LSE = mala.mala_fwd_prefill(Q, Kd, Vd, w.scale, tau, flags=flags, workspace=ws,
-                                   tile_mask=mask)
+    with mala.debug_margins(margin):
+        O, LSE = mala.mala_fwd_prefill(Q, Kd, Vd, w.scale, tau, flags=flags, workspace=ws,
+                                       tile_mask=mask)
     torch.cuda.synchronize()
     assert mala.read_device_error(ws) == 0
     mask = mask.cpu().numpy()
@@ -75,26 +61,31 @@ def run_prefill(mala, Qc, K, V, w, tau, flags=0):
     assert (mask[~legal] == 255).all() and np.isin(mask[legal], (0, 1)).all()
     st = mala.get_stats(ws)
     assert st["legal_tiles"] == legal.sum() and st["retained_tiles"] == (mask[legal] == 1).sum()
-    return O.float().cpu().numpy(), LSE.cpu().numpy(), mask
+    return (O.float().cpu().numpy(), LSE.cpu().numpy(), mask,
+            margin.view(B, H, Tq, Tk).cpu().numpy())
 
 
-def check_prefill(orc, mala, w, Qc, K, V, tau, units=None, flags=0):
-    O, LSE, mask = run_prefill(mala, Qc, K, V, w, tau, flags)
+def check_prefill(orc, mala, w, Qc, K, V, tau, units=None, flags=0, max_flips=0):
+    O, LSE, mask, gmargin = run_prefill(mala, Qc, K, V, w, tau, flags)
     B, Nq, H, d = Qc.shape
     Nk = K.shape[1]
     legal_all = prefill_legal(B, H, Nq, Nk)
     force = np.where(legal_all, mask.astype(np.int16), -1).astype(np.int8)
     oO, oLSE, _, omargin = orc.mala_prefill(Qc, K, V, w.scale, tau, units=units, force=force)
     legal = prefill_legal(B, H, Nq, Nk, units)
-    band = prefill_bands(Qc, K, w.scale, H // K.shape[2])
-    n, near, bad, worst = P.compare_masks(mask, omargin, band, legal)
-    assert bad == 0, f"{bad} tile decisions differ beyond the band (worst margin {worst})"
+    label = (f"prefill {w.structure} B{B} H{H}/{K.shape[2]} Nq{Nq} Nk{Nk} d{d} {w.dtype} "
+             f"tau={tau:g}" + (" always-test" if flags else ""))
+    row = {"flips": 0}
+    if tau > 0 or flags:
+        row = P.compare_decisions(label, "fp32" if w.dtype == "fp32" else "fwd", mask, gmargin,
+                                  omargin, legal, max_flips)
     rows = np.isfinite(oLSE)
-    P.check_output(O, oO, np.transpose(rows, (0, 2, 1)))
+    P.check_output(O, oO, np.transpose(rows, (0, 2, 1)), label)
     assert np.abs(LSE - oLSE)[rows].max() < P.LSE_ABS
     if tau == 0:
         assert (mask[legal_all] == 1).all()
-    return {"tiles": n, "near": near, "retained": float(mask[legal_all].mean())}
+    return {"tiles": int(legal.sum()), "flips": row["flips"],
+            "retained": float(mask[legal_all].mean())}
 
 
 @pytest.mark.parametrize("tau", [0.0, 1.0])
@@ -121,7 +112,7 @@ def test_prefill_aligned_chunk_equals_forward_tail_bitwise(mala):
     """With a 128-aligned offset the chunk's query blocks are the full forward's last
     blocks: same tiles, same order, same arithmetic -> identical bits."""
     w, Qc, K, V, Qf = chunk(1, 8, 2, 512, 1536, 128, "sink_band", seed=63)
-    Oc, Lc, Mc = run_prefill(mala, Qc, K, V, w, 1.0)
+    Oc, Lc, Mc, _ = run_prefill(mala, Qc, K, V, w, 1.0)
     Qd, Kd, Vd = (P.to_dev(x, "bf16") for x in (Qf, K, V))
     T = mala.n_tiles(1536)
     Mf = torch.full((1, 8, T, T), 255, dtype=torch.uint8, device="cuda")
@@ -216,7 +207,7 @@ def test_varlen_parity_with_oracle(orc, mala):
     O, LSE = O.float().cpu().numpy(), LSE.cpu().numpy()
     for s, (Qc, Ks, Vs, w) in enumerate(parts):
         # the GPU's decisions for this sequence (from its own prefill call) are replayed
-        _, _, mask = run_prefill(mala, Qc, Ks, Vs, w, 1.0)
+        _, _, mask, _ = run_prefill(mala, Qc, Ks, Vs, w, 1.0)
         legal = prefill_legal(1, H, Qc.shape[1], Ks.shape[1])
         force = np.where(legal, mask.astype(np.int16), -1).astype(np.int8)
         oO, oLSE, _, _ = orc.mala_prefill(Qc, Ks, Vs, scale, 1.0, force=force)

@@ -52,7 +52,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 def test_version_and_status_strings(lib):
     L = lib.lib()
-    assert L.mala_version() == 201
+    assert L.mala_version() == 202
     assert L.mala_status_string(0) == b"ok"
     assert L.mala_status_string(4) == b"device wait timed out"
 
@@ -200,3 +200,40 @@ def test_bench_two_ranks_gloo(tmp_path):
     assert out.returncode == 0, out.stderr[-2000:]
     found = sorted(re.findall(r"rank=\d seed=\d+ max=[\d.]+", out.stdout))
     assert found == ["rank=0 seed=3 max=11.0", "rank=1 seed=1003 max=11.0"], out.stdout
+
+
+def test_noalloc_decode_rejects_oversized_problems(lib):
+    """The size check of the allocation-free decode comes before any CUDA call: run on a
+    machine without a GPU only, with placeholder addresses that are never dereferenced."""
+    if torch.cuda.is_available():
+        pytest.skip("host-only check (placeholder addresses)")
+    L = lib.lib()
+    # 64 x 64 heads x 1024 splits of (128 + 1) floats is far beyond the fixed scratch
+    need = L.mala_decode_workspace_bytes(64, 64, 8, 131072, 128, 0, 1024)
+    assert need > 4 << 20
+    p = ctypes.c_void_p(1 << 20)
+    st = L.mala_decode_noalloc(p, p, p, p, p, 64, 64, 8, 131072, 128, 0, 0.1, 1.0, 1024, 0,
+                               None, None)
+    assert st == 5  # MALA_ERR_WORKSPACE
+
+
+def test_debug_margin_buffer_too_small_is_rejected_before_any_launch(lib):
+    """mala_set_debug: a call that needs more margin entries than registered returns
+    MALA_ERR_INVALID_ARG before any CUDA call (host only, placeholder addresses)."""
+    if torch.cuda.is_available():
+        pytest.skip("host-only check (placeholder addresses)")
+    L = lib.lib()
+    p = ctypes.c_void_p(16 * 1024)
+    dbg = lib.MalaDebug(16 * 1024, 3)  # 3 entries; a 2-block forward needs 1*2*2*2 = 8
+    assert L.mala_set_debug(ctypes.byref(dbg)) == 0
+    try:
+        assert L.mala_fwd(p, p, p, p, p, 1, 2, 1, 256, 128, 0, 0.1, 1.0, 0, None, 0, None,
+                          None) == 1
+        assert L.mala_bwd(p, p, p, p, p, p, p, p, p, 1, 2, 1, 256, 128, 0, 0.1, 1.0, 0, None, 0,
+                          None, None) == 1
+        assert L.mala_decode(p, p, p, p, p, 1, 2, 1, 1000, 128, 0, 0.1, 1.0, 1, 0, None, 0,
+                             None, None) == 1  # [1, 2, 8] = 16 entries
+    finally:
+        assert L.mala_set_debug(None) == 0
+    bad = lib.MalaDebug(16 * 1024 + 2, 8)  # misaligned buffer
+    assert L.mala_set_debug(ctypes.byref(bad)) == 1
