@@ -15,6 +15,7 @@ import ctypes
 import os
 import subprocess
 import threading
+import time
 
 import numpy as np
 
@@ -23,6 +24,20 @@ _SRC = os.path.join(_HERE, "mala_oracle.cpp")
 _LIB = os.path.join(_HERE, "libmala_oracle.so")
 _lock = threading.Lock()
 _lib = None
+
+# Wall-clock and process CPU seconds of the last oracle call, measured around the C call
+# alone (the Python-side array set-up is excluded); the bench's CPU baseline uses them.
+LAST_CALL = {"wall": 0.0, "cpu": 0.0}
+
+
+class _Timed:
+    def __enter__(self):
+        self.w, self.c = time.perf_counter(), time.process_time()
+
+    def __exit__(self, *exc):
+        LAST_CALL["wall"] = time.perf_counter() - self.w
+        LAST_CALL["cpu"] = time.process_time() - self.c
+        return False
 
 _f32p = np.ctypeslib.ndpointer(dtype=np.float32, flags="C_CONTIGUOUS")
 _f64p = np.ctypeslib.ndpointer(dtype=np.float64, flags="C_CONTIGUOUS")
@@ -58,6 +73,7 @@ def _load():
                                             ci, vp, vp, vp, vp, vp, vp, vp]
             lib.orc_mala_prefill.argtypes = [vp, vp, vp, ci, ci, ci, ci, ci, ci, cd, cd, ci, vp,
                                              ci, vp, vp, vp, vp, vp]
+            lib.orc_num_threads.restype = ctypes.c_int
             for name in ("orc_dense_fwd", "orc_dense_bwd", "orc_mala_fwd", "orc_mala_fwd_setsum",
                          "orc_mala_bwd", "orc_mala_decode", "orc_mala_prefill"):
                 getattr(lib, name).restype = ctypes.c_int
@@ -134,8 +150,9 @@ def mala_fwd(Q, K, V, scale, tau, blk=128, units=None, force=None):
     if force is not None:
         force = np.ascontiguousarray(force, dtype=np.int8)
         assert force.shape == (B, H, T, T)
-    rc = _load().orc_mala_fwd(_p(Q), _p(K), _p(V), B, H, Hkv, L, d, float(scale), float(tau), blk,
-                              _p(u), n, _p(force), _p(O), _p(LSE), _p(mask), _p(margin))
+    with _Timed():
+        rc = _load().orc_mala_fwd(_p(Q), _p(K), _p(V), B, H, Hkv, L, d, float(scale), float(tau), blk,
+                                  _p(u), n, _p(force), _p(O), _p(LSE), _p(mask), _p(margin))
     _check(rc, "mala_fwd")
     return O, LSE, mask, margin
 
@@ -156,9 +173,10 @@ def mala_prefill(Q, K, V, scale, tau, blk=128, units=None, force=None):
     if force is not None:
         force = np.ascontiguousarray(force, dtype=np.int8)
         assert force.shape == (B, H, Tq, Tk)
-    rc = _load().orc_mala_prefill(_p(Q), _p(K), _p(V), B, H, Hkv, Nq, Nk, d, float(scale),
-                                  float(tau), blk, _p(u), n, _p(force), _p(O), _p(LSE), _p(mask),
-                                  _p(margin))
+    with _Timed():
+        rc = _load().orc_mala_prefill(_p(Q), _p(K), _p(V), B, H, Hkv, Nq, Nk, d, float(scale),
+                                      float(tau), blk, _p(u), n, _p(force), _p(O), _p(LSE), _p(mask),
+                                      _p(margin))
     _check(rc, "mala_prefill")
     return O, LSE, mask, margin
 
@@ -198,9 +216,10 @@ def mala_bwd(Q, K, V, O, LSE, dO, scale, tau, blk=128, kv_units=None, q_units=No
     if force is not None:
         force = np.ascontiguousarray(force, dtype=np.int8)
         assert force.shape == (B, H, T, T)
-    rc = _load().orc_mala_bwd(_p(Q), _p(K), _p(V), _p(O), _p(LSE), _p(dO), B, H, Hkv, L, d,
-                              float(scale), float(tau), blk, _p(ku), nk, _p(qu), nq, _p(force),
-                              _p(dQ), _p(dK), _p(dV), _p(mask), _p(margin))
+    with _Timed():
+        rc = _load().orc_mala_bwd(_p(Q), _p(K), _p(V), _p(O), _p(LSE), _p(dO), B, H, Hkv, L, d,
+                                  float(scale), float(tau), blk, _p(ku), nk, _p(qu), nq, _p(force),
+                                  _p(dQ), _p(dK), _p(dV), _p(mask), _p(margin))
     _check(rc, "mala_bwd")
     return dQ, dK, dV, mask, margin
 
@@ -229,8 +248,14 @@ def mala_decode(q, K, V, scale, tau, num_splits, blk=128, units=None, force=None
     if force is not None:
         force = np.ascontiguousarray(force, dtype=np.int8)
         assert force.shape == (B, H, T)
-    rc = _load().orc_mala_decode(_p(q), _p(K), _p(V), B, H, Hkv, Nk, d, float(scale), float(tau),
-                                 blk, S, _p(u), n, _p(force), _p(O), _p(LSE), _p(mask),
-                                 _p(margin), _p(part_o), _p(part_z))
+    with _Timed():
+        rc = _load().orc_mala_decode(_p(q), _p(K), _p(V), B, H, Hkv, Nk, d, float(scale), float(tau),
+                                     blk, S, _p(u), n, _p(force), _p(O), _p(LSE), _p(mask),
+                                     _p(margin), _p(part_o), _p(part_z))
     _check(rc, "mala_decode")
     return O, LSE, mask, margin, part_o, part_z
+
+
+def num_threads() -> int:
+    """Threads the oracle's parallel loops use (OpenMP), i.e. the cores it occupies."""
+    return int(_load().orc_num_threads())

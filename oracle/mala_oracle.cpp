@@ -34,6 +34,10 @@
 #include <limits>
 #include <vector>
 
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
 namespace {
 
 const double kInf = std::numeric_limits<double>::infinity();
@@ -467,6 +471,16 @@ void prefill_block(const PDims& D, const float* Q, const float* K, const float* 
 extern "C" {
 
 int orc_version(void) { return 1; }
+
+// Threads the parallel loops below use (1 without OpenMP): the core count that the timed
+// CPU baseline reports.
+int orc_num_threads(void) {
+#ifdef _OPENMP
+  return omp_get_max_threads();
+#else
+  return 1;
+#endif
+}
 
 // Dense causal attention (FullAttn), rows of the listed (b, h, i) blocks of `blk`
 // rows (all rows when units == NULL).  O [B,L,H,d], LSE [B,H,L].

@@ -127,16 +127,16 @@ def format_report(rows) -> str:
     out = [r for r in rows if "o_raw_max" in r]
     if dec:
         lines.append("decision parity (margins in natural-log units; GPU vs fp64 oracle)")
-        lines.append(f"{'test':58s} {'tiles':>8s} {'kept':>6s} {'flips':>5s} {'max|dm|':>9s} "
+        lines.append(f"{'test':72s} {'tiles':>8s} {'kept':>6s} {'flips':>5s} {'max|dm|':>9s} "
                      f"{'p99.9|dm|':>9s} {'worst flip':>10s} {'min|m|':>9s}")
         for r in dec:
-            lines.append(f"{r['label'][:58]:58s} {r['tiles']:8d} {r['retained']:6.3f} "
+            lines.append(f"{r['label'][:72]:72s} {r['tiles']:8d} {r['retained']:6.3f} "
                          f"{r['flips']:5d} {r['max_err']:9.2e} {r['p999_err']:9.2e} "
                          f"{r['worst_flip']:10.2e} {r['min_abs_margin']:9.2e}")
     if out:
         lines.append("outputs (O vs oracle): scaled max |dO|/max(1,|O|), raw max, mean, "
                      "elements over 1e-2")
         for r in out:
-            lines.append(f"{r['label'][:58]:58s} {r['o_scaled_max']:9.2e} {r['o_raw_max']:9.2e} "
+            lines.append(f"{r['label'][:72]:72s} {r['o_scaled_max']:9.2e} {r['o_raw_max']:9.2e} "
                          f"{r['o_mean']:9.2e} {r['o_over_1e-2']:6d}/{r['o_elems']}")
     return "\n".join(lines)

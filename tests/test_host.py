@@ -202,6 +202,83 @@ def test_bench_two_ranks_gloo(tmp_path):
     assert found == ["rank=0 seed=3 max=11.0", "rank=1 seed=1003 max=11.0"], out.stdout
 
 
+_SHARD_CHILD = r"""
+import os, sys
+sys.path.insert(0, {root!r})
+import numpy as np
+import bench
+import oracle
+d = bench.Dist().init("gloo")
+r, n = d.rank, d.world
+w, inp = bench.synth.small_training(B=1, H=8, Hkv=4, L=384, d=32, structure="peaked", seed=5)
+ws, part = bench.shard_training(w, inp, r, n)
+O, LSE, mask, _ = oracle.mala_fwd(part["Q"], part["K"], part["V"], w.scale, 1.0)
+dQ, dK, dV, bmask, _ = oracle.mala_bwd(part["Q"], part["K"], part["V"], O, LSE, part["dO"],
+                                       w.scale, 1.0)
+wd = bench.synth.Workload("shard_decode", 2, 8, 4, 1000, 32, "bf16", "planted", 6, decode=True)
+dec = bench.synth.make_decode(wd)
+wds, dpart = bench.shard_decode(wd, dec, r, n)
+Od, Ld, dmask, _, _, _ = oracle.mala_decode(dpart["q"], dpart["K"], dpart["V"], wd.scale, 1.0, 3)
+np.savez({out!r} + f"/rank{{r}}.npz", O=O, LSE=LSE, mask=mask, dQ=dQ, dK=dK, dV=dV,
+         bmask=bmask, Od=Od, Ld=Ld, dmask=dmask, H=ws.H, Hkv=ws.H_kv)
+v = d.max(10.0 + r)
+d.barrier()
+print(f"rank={{r}} heads={{ws.H}}/{{ws.H_kv}} max={{v}}", flush=True)
+d.close()
+"""
+
+
+def test_head_sharding_partition():
+    sys.path.insert(0, ROOT)
+    import bench
+
+    for world in (1, 2, 4, 8):
+        got = [bench.head_shard(32, 8, r, world) for r in range(world)]
+        # contiguous, disjoint, covering; query heads follow their KV heads (G = 4)
+        assert got[0][0] == 0 and got[-1][1] == 8 and got[-1][3] == 32
+        for (g0, g1, h0, h1), nxt in zip(got, got[1:] + [None]):
+            assert g1 - g0 == 8 // world and (h0, h1) == (4 * g0, 4 * g1)
+            if nxt:
+                assert nxt[0] == g1 and nxt[2] == h1
+    with pytest.raises(ValueError):
+        bench.head_shard(32, 8, 0, 3)
+
+
+def test_head_sharded_ranks_reproduce_the_unsharded_problem_gloo(tmp_path):
+    """Two gloo ranks each run the oracle on their head shard of one problem; the shards,
+    put back together along the head axis, equal the unsharded results exactly (every head
+    is independent, so sharding changes nothing), and the timing reduction is a max."""
+    import oracle
+    from mass_adaptive_sparse_fwd_b200 import synth
+
+    script = tmp_path / "child.py"
+    script.write_text(_SHARD_CHILD.format(root=ROOT, out=str(tmp_path)))
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node=2",
+           "--master-addr", "127.0.0.1", "--master-port", "29541", str(script)]
+    out = subprocess.run(cmd, capture_output=True, text=True, timeout=300)
+    assert out.returncode == 0, out.stderr[-2000:]
+    found = sorted(re.findall(r"rank=\d heads=\d+/\d+ max=[\d.]+", out.stdout))
+    assert found == ["rank=0 heads=4/2 max=11.0", "rank=1 heads=4/2 max=11.0"], out.stdout
+    parts = [np.load(tmp_path / f"rank{r}.npz") for r in range(2)]
+    w, inp = synth.small_training(B=1, H=8, Hkv=4, L=384, d=32, structure="peaked", seed=5)
+    O, LSE, mask, _ = oracle.mala_fwd(inp["Q"], inp["K"], inp["V"], w.scale, 1.0)
+    dQ, dK, dV, bmask, _ = oracle.mala_bwd(inp["Q"], inp["K"], inp["V"], O, LSE, inp["dO"],
+                                           w.scale, 1.0)
+    cat = lambda k, ax: np.concatenate([p[k] for p in parts], axis=ax)
+    np.testing.assert_array_equal(cat("O", 2), O)
+    np.testing.assert_array_equal(cat("LSE", 1), LSE)
+    np.testing.assert_array_equal(cat("mask", 1), mask)
+    np.testing.assert_array_equal(cat("bmask", 1), bmask)
+    for k, ref in (("dQ", dQ), ("dK", dK), ("dV", dV)):
+        np.testing.assert_array_equal(cat(k, 2), ref)
+    wd = synth.Workload("shard_decode", 2, 8, 4, 1000, 32, "bf16", "planted", 6, decode=True)
+    dec = synth.make_decode(wd)
+    Od, Ld, dmask, _, _, _ = oracle.mala_decode(dec["q"], dec["K"], dec["V"], wd.scale, 1.0, 3)
+    np.testing.assert_array_equal(cat("Od", 1), Od)
+    np.testing.assert_array_equal(cat("Ld", 1), Ld)
+    np.testing.assert_array_equal(cat("dmask", 1), dmask)
+
+
 def test_noalloc_decode_rejects_oversized_problems(lib):
     """The size check of the allocation-free decode comes before any CUDA call: run on a
     machine without a GPU only, with placeholder addresses that are never dereferenced."""
