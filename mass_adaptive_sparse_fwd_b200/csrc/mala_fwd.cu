@@ -14,21 +14,25 @@
 // different lengths (varlen) gives every unit its own sequence's row bases, length and
 // offset through a host-built table (FwdParams::vtab).
 //
-// Warp roles (384 threads):
-//   warp 0      TMA producer: Q of both slots, then K_j and V_j per key block into a
-//               ring of NS stages.  V is fetched together with K (see below).
-//   warp 1      TMEM owner and UMMA issuer: S_s = Q_s K_j^T (SS, both K-major) into
-//               TMEM, and O_s += P_s V_j (TS: P in TMEM, V MN-major) for retained tiles.
-//   warps 4-7   softmax / retention test for slot 0 (thread = query row = TMEM lane)
-//   warps 8-11  same for slot 1
+// Warp roles (576 threads):
+//   warp 0       TMA producer: Q of both slots, then K_j and V_j per key block into a
+//                ring of NS stages.  V is fetched together with K (see below).
+//   warp 1       TMEM owner and UMMA issuer: S_s = Q_s K_j^T (SS, both K-major) into
+//                TMEM, and O_s += P_s V_j (TS: P in TMEM, V MN-major) for retained tiles.
+//   warps 2-9    softmax / retention test for slot 0: thread = query row = TMEM lane,
+//                warps 2-5 on keys 0..63 of the tile and warps 6-9 on keys 64..127; the
+//                two halves exchange their row maxima and shares of the row sum through
+//                shared memory once per tile
+//   warps 10-17  same for slot 1
 // TMEM columns: S_0 [0,128), S_1 [128,256), O_0 [256,256+D), O_1 [256+D, 256+2D).
-// P_s (bf16, packed in pairs) overwrites the first 64 columns of S_s.
+// P_s (bf16, packed in pairs) overwrites, in each half, the first 32 of its 64 columns of
+// S_s: keys 0..63 in columns [0, 32), keys 64..127 in columns [64, 96).
 //
 // Retention test (Eq. 3) per row q in the log2 domain: with the running state
 // (m, l) of retained tiles, log2 Z = m + log2 l.  A row keeps the tile if l == 0
 // (its first legal tile) or rowmax(S) * scale * log2(e) >= m + log2(l) + log2(tau/L_q),
 // L_q = position + 1; rows with no legal key in the tile (above the diagonal, or q >= L) do
-// not vote.  The tile is retained if any row keeps it (bar.red.or over the 128
+// not vote.  The tile is retained if any row keeps it (bar.red.or over the slot's 256
 // threads).  A skipped tile leaves m, l and O untouched and costs only the QK^T MMA,
 // the TMEM load of S and the row maxima: no exponentials, no P store, no PV MMA.
 //
@@ -60,7 +64,7 @@ struct FwdCfg {
   static constexpr int TILE_BYTES = kTile * D * 2;       // one 128 x D bf16 tile
   static constexpr int BOXES = D / 64;                   // 64-column TMA boxes per tile
   static constexpr int SMEM = 2 * TILE_BYTES + 2 * NS * TILE_BYTES + 1024;
-  static constexpr int THREADS = 384;
+  static constexpr int THREADS = 576;  // warps 0-1 TMA / MMA, warps 2-17 softmax
 };
 
 struct FwdShared {
@@ -73,6 +77,10 @@ struct FwdShared {
   uint32_t dec[2];
   uint32_t tmem_base;
   uint32_t abort_flag;
+  // per slot and key-column half: the half's raw row maximum of the current tile and its
+  // share of the running row sum, exchanged once per tile
+  float xmax[2][2][128];
+  float xsum[2][2][128];
 };
 
 static_assert(FwdCfg<128>::SMEM + sizeof(FwdShared) <= 232448, "forward smem budget");
@@ -130,7 +138,7 @@ __device__ __forceinline__ Unit decode_unit(const FwdParams& p, int u) {
 }
 
 template <int D, bool kScreen>
-__global__ void __launch_bounds__(384, 1)
+__global__ void __launch_bounds__(576, 1)
     mala_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
   using C = FwdCfg<D>;
@@ -152,10 +160,10 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(&sh.q_full[s], 1);
       mbar_init(&sh.q_empty[s], 1);
       mbar_init(&sh.s_full[s], 1);
-      mbar_init(&sh.p_full[s], 128);
+      mbar_init(&sh.p_full[s], 8);  // one arrival per softmax warp of the slot
       mbar_init(&sh.o_done[s], 1);
       mbar_init(&sh.sched_full[s], 1);
-      mbar_init(&sh.sched_empty[s], 1 + 256);
+      mbar_init(&sh.sched_empty[s], 1 + 512);
     }
     for (int st = 0; st < NS; ++st) {
       mbar_init(&sh.k_full[st], 1);
@@ -287,8 +295,8 @@ __global__ void __launch_bounds__(384, 1)
                 break;
               const uint32_t va = smem_u32(sV + st * C::TILE_BYTES);
 #pragma unroll
-              for (int kk = 0; kk < 8; ++kk)
-                umma_ts(tb + 256 + s * D, tb + s * 128 + kk * 8,
+              for (int kk = 0; kk < 8; ++kk)  // P of keys 16 kk .. (see the softmax's pass 2)
+                umma_ts(tb + 256 + s * D, tb + s * 128 + (kk >> 2) * 64 + (kk & 3) * 8,
                         sdesc_sw128(va + kk * 2048, 16384, 1024), id_pv,
                         (o_started[s] || kk > 0) ? 1u : 0u);
               o_started[s] = true;
@@ -320,23 +328,32 @@ __global__ void __launch_bounds__(384, 1)
       fin.budget_ns = kTeardownBudgetNs;
       mbar_wait(&sh.final_bar, 0, fin, 17);
     }
-  } else if (warp >= 4) {
+  } else if (warp >= 2) {
     // ------------------------------------------------------------------ softmax
-    const int s = (warp - 4) >> 2;          // slot
+    // warps 2..17: slot s = (warp - 2) / 8 and key-column half hf = ((warp - 2) / 4) % 2;
+    // the warp reaches TMEM lanes 32 (warp % 4) .. + 31 (four consecutive warps cover the
+    // 128 rows), so thread = query row r and each half handles 64 of the tile's 128 keys
+    const int wsm = warp - 2;
+    const int s = wsm >> 3;                 // slot
+    const int hf = (wsm >> 2) & 1;          // key-column half
     const int wq = warp & 3;                // TMEM lane quarter
     const int r = wq * 32 + lane;           // row within the tile
+    const int c0 = hf * 64;                 // this half's key columns [c0, c0 + 64)
+    constexpr int DH = D / 2;               // this half's head-dim columns of O
+    const uint32_t bar_slot = 1 + s;        // named barrier of the slot's 256 threads
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
     const uint32_t tS = tb + s * 128 + lane_off;
-    const uint32_t tO = tb + 256 + s * D + lane_off;
+    const uint32_t tO = tb + 256 + s * D + lane_off + hf * DH;
     const float NEG_INF = -INFINITY;
     uint32_t ns = 0, npv = 0;  // tiles tested / retained by this slot (also the stats)
     bool ok = true;
     for (uint32_t k = 0; ok; ++k) {
       const int ring = k & 1;
-      // every exit of this loop is decided right after a warpgroup barrier, so that the
-      // 128 threads of the slot always leave together
+      // every exit of this loop is decided by a barrier reduction over the slot's 256
+      // threads (a failed wait, or the abort flag seen by any of them), so that they
+      // always leave together
       const bool got = mbar_wait(&sh.sched_full[ring], (k >> 1) & 1, ast, 20);
-      if (named_bar_or(1 + s, 128, !got) || *ast.flag) { ok = false; break; }
+      if (named_bar_or(bar_slot, 256, !got || *ast.flag)) { ok = false; break; }
       const int u = sh.sched_ring[ring];
       mbar_arrive(&sh.sched_empty[ring]);
       if (u >= p.n_units) break;
@@ -348,6 +365,8 @@ __global__ void __launch_bounds__(384, 1)
       // L_q = position + 1 (the position is q in a full forward, off + q in a chunk)
       const float thr2 =
           kScreen ? (p.log2_tau - __log2f(static_cast<float>(w.off + q + 1))) : NEG_INF;
+      // m2: running maximum (log2 units, the same in both halves); l: this half's share of
+      // the running sum (the row's sum is the two halves' shares added)
       float m2 = NEG_INF, l = 0.f;
       const uint32_t npv_unit0 = npv;
       const int jl = last_key_tile(w);
@@ -355,93 +374,90 @@ __global__ void __launch_bounds__(384, 1)
       const int n = jl + 1;
       for (int t = 0; t < n; ++t) {
         const int j = jl - t;
-        // A failed wait never leaves the loop before the next named barrier of the
-        // warpgroup: the abort flag is set and checked right after the vote.
-        const bool got = mbar_wait(&sh.s_full[s], ns & 1, ast, 21);
+        const bool got = mbar_wait_warp(&sh.s_full[s], ns & 1, ast, 21);
         ++ns;
         tc_fence_after();
-        // pass 1: row maximum of the raw scores (the scale is positive, so it commutes
-        // with max), 64 columns at a time; only tiles that reach past the block's first
-        // position (the diagonal tile, and its neighbour when the chunk offset is not a
-        // multiple of 128) and rows past the end need masking: key c is legal for row r
-        // iff c <= lim = position - 128 j
-        const bool warp_ok = __all_sync(0xffffffffu, got);
+        // pass 1: this half's row maximum of the raw scores (the scale is positive, so it
+        // commutes with max); only tiles that reach past the block's first position and
+        // rows past the end need masking: key c is legal for row r iff c <= lim
         const bool masked = (j * kTile + kTile - 1 > pos0) || !valid;
         const int lim = valid ? (pos0 + r - j * kTile) : -1;
         float rraw = NEG_INF;
-        if (warp_ok) {
+        if (got) {
 #pragma unroll
-          for (int hh = 0; hh < 2; ++hh) {
-            uint32_t v[2][32];
-            tmem_ld32(tS + hh * 64, v[0]);
-            tmem_ld32(tS + hh * 64 + 32, v[1]);
+          for (int a = 0; a < 2; ++a) {  // 32 columns at a time (register budget)
+            uint32_t v[32];
+            tmem_ld32(tS + c0 + a * 32, v);
             tmem_wait_ld();
             if (masked) {
 #pragma unroll
-              for (int a = 0; a < 2; ++a)
-#pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                  const int col = hh * 64 + a * 32 + e;
-                  rraw = fmaxf(rraw, col <= lim ? __uint_as_float(v[a][e]) : NEG_INF);
-                }
+              for (int e = 0; e < 32; ++e) {
+                const int col = c0 + a * 32 + e;
+                rraw = fmaxf(rraw, col <= lim ? __uint_as_float(v[e]) : NEG_INF);
+              }
             } else {
-              // four independent three-input max chains (a single chain would serialise
-              // 64 dependent max operations per 64 columns)
+              // four independent three-input max chains
               float r0 = rraw, r1 = NEG_INF, r2 = NEG_INF, r3 = NEG_INF;
 #pragma unroll
-              for (int a = 0; a < 2; ++a)
-#pragma unroll
-                for (int e = 0; e < 32; e += 8) {
-                  r0 = fmax3(r0, __uint_as_float(v[a][e]), __uint_as_float(v[a][e + 1]));
-                  r1 = fmax3(r1, __uint_as_float(v[a][e + 2]), __uint_as_float(v[a][e + 3]));
-                  r2 = fmax3(r2, __uint_as_float(v[a][e + 4]), __uint_as_float(v[a][e + 5]));
-                  r3 = fmax3(r3, __uint_as_float(v[a][e + 6]), __uint_as_float(v[a][e + 7]));
-                }
+              for (int e = 0; e < 32; e += 8) {
+                r0 = fmax3(r0, __uint_as_float(v[e]), __uint_as_float(v[e + 1]));
+                r1 = fmax3(r1, __uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
+                r2 = fmax3(r2, __uint_as_float(v[e + 4]), __uint_as_float(v[e + 5]));
+                r3 = fmax3(r3, __uint_as_float(v[e + 6]), __uint_as_float(v[e + 7]));
+              }
               rraw = fmaxf(fmaxf(r0, r1), fmaxf(r2, r3));
             }
           }
         }
+        // exchange with the other half: its row maximum of this tile and its share of the
+        // running sum.  The barrier also orders every S load of the tile before the P
+        // stores below, and the previous tile's reads of the exchange slots before these
+        // writes (they come after that tile's vote / this barrier's predecessor).
+        sh.xmax[s][hf][r] = rraw;
+        sh.xsum[s][hf][r] = l;
+        if (named_bar_or(bar_slot, 256, !got || *ast.flag)) { ok = false; break; }
+        rraw = fmaxf(rraw, sh.xmax[s][hf ^ 1][r]);
+        const float lrow = l + sh.xsum[s][hf ^ 1][r];
         const float rmax = rraw * p.scale_log2;
         bool keep = true;
         if (kScreen) {
-          const float cut = m2 + __log2f(l) + thr2;
-          const bool mine = (rmax != NEG_INF) && (l == 0.f || rmax >= cut);
-          keep = named_bar_or(1 + s, 128, mine);
-          if (p.tile_margin) {
+          const float cut = m2 + __log2f(lrow) + thr2;
+          const bool mine = (rmax != NEG_INF) && (lrow == 0.f || rmax >= cut);
+          keep = named_bar_or(bar_slot, 256, mine);
+          if (p.tile_margin && hf == 0) {
             // debug: the tile's margin max_q (rowmax - cut) in natural-log units (+inf for
             // a row's first retained tile, -inf for rows without a legal key)
-            float x = (rmax == NEG_INF) ? NEG_INF : (l == 0.f ? INFINITY : rmax - cut);
+            float x = (rmax == NEG_INF) ? NEG_INF : (lrow == 0.f ? INFINITY : rmax - cut);
             x = warp_max_f32(x);
             if (lane == 0)
               atomic_max_f32(p.tile_margin + ((static_cast<size_t>(w.b) * p.H + h) * p.T + w.i) *
                                                  p.Tk + j,
                              x * kLn2);
           }
-          if (*ast.flag) { ok = false; break; }
         }
-        if (p.tile_mask && r == 0)
+        if (p.tile_mask && r == 0 && hf == 0)
           p.tile_mask[((static_cast<size_t>(w.b) * p.H + h) * p.T + w.i) * p.Tk + j] = keep ? 1 : 0;
         if (!keep) {
-          if (r == 0) sh.dec[s] = 0;
+          if (r == 0 && hf == 0) sh.dec[s] = 0;
           tc_fence_before();
-          mbar_arrive(&sh.p_full[s]);
+          warp_arrive(&sh.p_full[s]);
           continue;
         }
-        // lazy running-max update
+        // lazy running-max update (identical in both halves)
         float m_new = m2;
         bool rescale = false;
         if (rmax > m2 + 8.0f) {
           m_new = rmax;
-          rescale = (l > 0.f);
+          rescale = (lrow > 0.f);
         }
         const float m_use = (m_new == NEG_INF) ? 0.f : m_new;
         const float alpha = rescale ? fast_exp2(m2 - m_new) : 1.f;
         if (__any_sync(0xffffffffu, rescale) &&
             // the previous PV of this slot must have landed before O is touched
-            __all_sync(0xffffffffu, mbar_wait(&sh.o_done[s], (npv - 1) & 1, ast, 22))) {
+            mbar_wait_warp(&sh.o_done[s], (npv - 1) & 1, ast, 22)) {
           tc_fence_after();
 #pragma unroll
-          for (int cc = 0; cc < D / 32; ++cc) {
+          for (int cc = 0; cc < DH / 32; ++cc) {
             uint32_t o[32];
             tmem_ld32(tO + cc * 32, o);
             tmem_wait_ld();
@@ -450,21 +466,22 @@ __global__ void __launch_bounds__(384, 1)
             tmem_st32(tO + cc * 32, o);
           }
         }
-        // pass 2: P = exp2(s * scale * log2(e) - m), 32 keys at a time, packed into the
-        // first 64 columns of the same TMEM region (each store lands on columns this
-        // thread has already read)
+        // pass 2: P = exp2(s * scale * log2(e) - m) over this half's 64 keys, 32 at a
+        // time, packed into the first 32 columns of the half's own 64 (each store lands on
+        // columns this thread has already read); the PV MMA reads keys 0..63 from columns
+        // [0, 32) and keys 64..127 from columns [64, 96) of the slot's S region
         float ps0 = 0.f, ps1 = 0.f;  // two independent partial sums
 #pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
+        for (int cc = 0; cc < 2; ++cc) {
           uint32_t v[32];
-          if (warp_ok) {
-            tmem_ld32(tS + cc * 32, v);
+          if (got) {
+            tmem_ld32(tS + c0 + cc * 32, v);
             tmem_wait_ld();
           }
           if (masked) {
 #pragma unroll
             for (int e = 0; e < 32; ++e)
-              if (cc * 32 + e > lim) v[e] = 0xff800000u;  // -inf: P = 0
+              if (c0 + cc * 32 + e > lim) v[e] = 0xff800000u;  // -inf: P = 0
           }
           uint32_t pk[16];
 #pragma unroll
@@ -474,28 +491,33 @@ __global__ void __launch_bounds__(384, 1)
             if (e & 1) ps1 += p0 + p1; else ps0 += p0 + p1;
             pk[e] = pack_bf16(p0, p1);
           }
-          tmem_st16(tS + cc * 16, pk);
+          tmem_st16(tS + c0 + cc * 16, pk);
         }
         tmem_wait_st();
-        const float psum = ps0 + ps1;
-        l = l * alpha + psum;
+        l = l * alpha + (ps0 + ps1);
         m2 = m_new;
-        if (r == 0) sh.dec[s] = 1;
+        if (r == 0 && hf == 0) sh.dec[s] = 1;
         tc_fence_before();
-        mbar_arrive(&sh.p_full[s]);
+        warp_arrive(&sh.p_full[s]);
         ++npv;
       }
       if (!ok) break;
-      // epilogue: O = acc / l, LSE = (m + log2 l) * ln 2
+      // epilogue: the row's sum from both halves (the exchange slots were last read before
+      // the last tile's vote), then O = acc / l on this half's head-dim columns and
+      // LSE = (m + log2 l) ln 2
+      sh.xsum[s][hf][r] = l;
+      named_bar_sync(bar_slot, 256);
+      const float lrow = l + sh.xsum[s][hf ^ 1][r];
       bool o_ready = true;
-      if (npv > npv_unit0) o_ready = mbar_wait(&sh.o_done[s], (npv - 1) & 1, ast, 23);
-      if (!__all_sync(0xffffffffu, o_ready)) continue;  // aborting: the next vote exits
+      if (npv > npv_unit0) o_ready = mbar_wait_warp(&sh.o_done[s], (npv - 1) & 1, ast, 23);
+      if (!o_ready) continue;  // aborting: the next barrier reduction exits (no barrier below)
       tc_fence_after();
-      const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
+      const float inv_l = (lrow > 0.f) ? 1.f / lrow : 0.f;
       __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.O) +
-                            ((static_cast<size_t>(w.b) * p.Lrows + w.qrow0 + q) * p.H + h) * D;
+                            ((static_cast<size_t>(w.b) * p.Lrows + w.qrow0 + q) * p.H + h) * D +
+                            hf * DH;
 #pragma unroll
-      for (int cc = 0; cc < D / 32; ++cc) {
+      for (int cc = 0; cc < DH / 32; ++cc) {
         uint32_t o[32];
         tmem_ld32(tO + cc * 32, o);
         tmem_wait_ld();
@@ -511,11 +533,12 @@ __global__ void __launch_bounds__(384, 1)
           }
         }
       }
-      if (valid)
-        p.LSE[(static_cast<size_t>(w.b) * p.H + h) * p.Lrows + w.qrow0 + q] = (m2 + __log2f(l)) * kLn2;
+      if (valid && hf == 0)
+        p.LSE[(static_cast<size_t>(w.b) * p.H + h) * p.Lrows + w.qrow0 + q] =
+            (m2 + __log2f(lrow)) * kLn2;
       tc_fence_before();
     }
-    if (r == 0) stats_add(p.stats, ns, npv, 0);
+    if (r == 0 && hf == 0) stats_add(p.stats, ns, npv, 0);
   }
 
   tc_fence_before();
