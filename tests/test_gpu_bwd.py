@@ -167,9 +167,13 @@ def test_bwd_prev_token_skips(orc, mala):
 
 
 @pytest.mark.slow
-def test_bwd_prevtok32k_sampled(orc, mala):
+@pytest.mark.parametrize("tau", [1.0, 0.0])
+def test_bwd_prevtok32k_sampled(orc, mala, tau):
+    """Concentrated states at 32K: the skip regime at tau = 1 and the dense path on the same
+    extreme scores (one dominant key per row) at tau = 0."""
     w = synth.WORKLOADS["prevtok32k"]
     T = w.L // 128
-    st = check_bwd(orc, mala, w, synth.make_training(w), 1.0,
+    st = check_bwd(orc, mala, w, synth.make_training(w), tau,
                    kv_units=[(0, 5, T - 3), (0, 0, 7)], q_units=[(0, 31, T - 1), (0, 2, 40)])
-    assert st["bwd_retained"] < 0.05
+    if tau > 0:
+        assert st["bwd_retained"] < 0.05
