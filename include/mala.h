@@ -167,8 +167,9 @@ mala_status mala_decode(const void* q, const void* Kc, const void* Vc, void* O, 
  *   num_splits = 0 the split rule keeps B * H_kv * S <= 296 whenever B * H_kv <= 296, so
  *   the scratch is at most 296 * (H / H_kv) * (d + 1) * 4 bytes plus a small header:
  *   every bf16 decode (groups of up to 8) of such a batch fits.
- *   The first call on a device looks up the array's device address (once per device,
- *   with that device current); make that first call before any stream capture.
+ *   The first call on a device looks up the array's device address (once per device and
+ *   driver context, with that device current; again after the context was recreated, e.g.
+ *   by cudaDeviceReset); make that first call before any stream capture.
  *   All calls on a device share the array: calls whose work overlaps on the GPU (two
  *   streams at once) race and must be serialised by the caller.  Device-side wait
  *   timeouts are recorded in the internal array and are not reported by this call.
