@@ -98,6 +98,7 @@ struct BwdShared {
   alignas(16) float dsum[2][64];
   int sched_ring[2];
   uint32_t dec;      // decision of the current tile (1 = retained)
+  uint32_t abort_seen[2];  // the abort flag as seen before a tile's vote (by tile parity)
   uint32_t dq_flag[2];
   uint32_t acc_valid;  // the unit retained at least one tile (dK / dV were written)
   uint32_t tmem_base;
@@ -382,7 +383,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     for (uint32_t k = 0; ok; ++k) {
       const int ring = k & 1;
       const bool got = mbar_wait(&sh.sched_full[ring], (k >> 1) & 1, ast, 20);
-      if (named_bar_or(1, 256, !got) || *ast.flag) { ok = false; break; }
+      // exits are decided by barrier reductions, so both softmax warpgroups leave together
+      if (named_bar_or(1, 256, !got || *ast.flag)) { ok = false; break; }
       const int u = sh.sched_ring[ring];
       mbar_arrive(&sh.sched_empty[ring]);
       if (u >= p.n_units) break;
@@ -471,6 +473,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 }
               }
           }
+          // the abort flag as one thread saw it before the vote: every thread reads the same
+          // copy after the barrier, so the exit below is uniform (the slot is rewritten two
+          // tiles later, after every reader has passed the next vote)
+          if (tid == 128) sh.abort_seen[ntile & 1] = *ast.flag;
           keep = named_bar_or(1, 256, ymax >= 0.f);
           if (p.tile_margin) {
             // debug: the tile's margin max over legal entries of log P - log(tau / L_q),
@@ -481,10 +487,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                                  w.j,
                              x * kLn2);
           }
+          if (sh.abort_seen[ntile & 1]) { ok = false; break; }
         } else {
-          named_bar_sync(1, 256);  // every S^T load done before P overwrites it
+          // every S^T load done before P overwrites it; the reduction decides the exit
+          if (named_bar_or(1, 256, *ast.flag != 0)) { ok = false; break; }
         }
-        if (*ast.flag) { ok = false; break; }
         if (p.tile_mask && tid == 128)
           p.tile_mask[((static_cast<size_t>(w.b) * p.H + h) * p.T + i) * p.T + w.j] = keep ? 1 : 0;
         if (!keep) {
@@ -567,7 +574,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     for (uint32_t k = 0; ok; ++k) {
       const int ring = k & 1;
       const bool got = mbar_wait(&sh.sched_full[ring], (k >> 1) & 1, ast, 30);
-      if (named_bar_or(4, 128, !got) || *ast.flag) { ok = false; break; }
+      if (named_bar_or(4, 128, !got || *ast.flag)) { ok = false; break; }
       const int u = sh.sched_ring[ring];
       mbar_arrive(&sh.sched_empty[ring]);
       if (u >= p.n_units) break;
