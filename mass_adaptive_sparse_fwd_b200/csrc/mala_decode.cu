@@ -99,10 +99,6 @@ struct DecShared {
   float rsum[2][8][8];
   uint32_t last_flag;
   uint32_t abort_flag;
-  // the abort flag as thread 0 saw it just before a per-tile barrier, by barrier parity:
-  // every consumer reads the same copy after the barrier, so all leave together (a slot is
-  // rewritten two barriers later, after every reader has passed the next one)
-  uint32_t abort_seen[2];
 };
 
 static_assert(DecCfg<128>::SMEM + sizeof(DecShared) <= 232448, "decode smem budget");
@@ -270,7 +266,6 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, 1)
     const float NEG_INF = -INFINITY;
     const uint32_t sKa = smem_u32(sK), sVa = smem_u32(sV);
     uint32_t kc = 0, vc = 0, n_glob = 0;
-    uint32_t nbar = 0;  // per-tile barriers passed (selects the abort_seen slot)
     uint32_t st_legal = 0, st_ret = 0;  // call statistics (thread 0)
     bool ok = true;
     // zero the padded heads of P once (rows >= G are never written again)
@@ -378,9 +373,7 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, 1)
             sh.rsum[rb][warp][lane * 2] = ps_prev[0];
             sh.rsum[rb][warp][lane * 2 + 1] = ps_prev[1];
           }
-          if (tid == 0) sh.abort_seen[nbar & 1] = *ast.flag;
-          named_bar_sync(1, NT);
-          if (sh.abort_seen[nbar++ & 1]) { ok = false; break; }  // the same copy for all
+          if (named_bar_or(1, NT, *ast.flag != 0)) { ok = false; break; }  // uniform exit
           #pragma unroll
           for (int hs = 0; hs < HS; ++hs)
             close_prev<CW>(sh.rsum[rb], dw, dh + 4 * hs, mnew_prev[hs], alpha_prev[hs],
@@ -464,9 +457,7 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, 1)
             sh.rsum[rb][warp][lane * 2] = ps_prev[0];
             sh.rsum[rb][warp][lane * 2 + 1] = ps_prev[1];
           }
-          if (tid == 0) sh.abort_seen[nbar & 1] = *ast.flag;
-          named_bar_sync(1, NT);
-          if (sh.abort_seen[nbar++ & 1]) { ok = false; break; }  // the same copy for all
+          if (named_bar_or(1, NT, *ast.flag != 0)) { ok = false; break; }  // uniform exit
           #pragma unroll
           for (int hs = 0; hs < HS; ++hs)
             close_prev<CW>(sh.rsum[rb], dw, dh + 4 * hs, mnew_prev[hs], alpha_prev[hs],
