@@ -28,12 +28,10 @@ def pytest_terminal_summary(terminalreporter):
         terminalreporter.write_line("")
         for line in parity.format_report(parity.REPORT).splitlines():
             terminalreporter.write_line(line)
-        try:
+        # optional machine-readable copy (MALA_PARITY_REPORT=<path.json>)
+        path = os.environ.get("MALA_PARITY_REPORT")
+        if path:
             import json
 
-            out = os.path.join(ROOT, "gpurun_out")
-            if os.path.isdir(out):
-                with open(os.path.join(out, "parity_report.json"), "w") as f:
-                    json.dump(parity.REPORT, f, indent=1)
-        except OSError:
-            pass
+            with open(path, "w") as f:
+                json.dump(parity.REPORT, f, indent=1)

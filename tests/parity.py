@@ -21,9 +21,9 @@ Tolerances:
       - consequently a decision may differ from the oracle's only where the oracle's
         margin is within MARGIN_ERR of the threshold; the number of such flips is
         recorded and asserted per test.
-    The 1e-6 band that was asked for lies below the fp32 rounding of the quantities
+    A 1e-6 band around the threshold would lie below the fp32 rounding of the quantities
     compared here (scores of magnitude 10-50, log-normalisers of magnitude 10-30,
-    thresholds log(tau / L_q) near -10), so the measured bound is the honest one.
+    thresholds log(tau / L_q) near -10), so the bound is set from the measured error.
 """
 
 from __future__ import annotations
