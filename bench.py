@@ -865,6 +865,95 @@ def profile_case(case: str):
                       "O_decode": float(Od.float().abs().mean())}), flush=True)
 
 
+SWEEP_LENGTHS = (1024, 2048, 4096, 8192, 16384, 32768, 65536, 131072)
+
+
+def run_sweep(args):
+    """Operator latency and peak memory across sequence lengths (the page's operator
+    benchmark, App. C.5 "Operator Latency and Memory Setup": batch 1, lengths 1K-128K,
+    25 warm-up and 100 timed iterations, peak per-rank allocation).  The shape is one
+    rank's share of a 64-query-head / 8-KV-head model under 8-way head sharding (H=8,
+    H_kv=1, d=128; the sharded ranks run independent problems of this shape), on the
+    sink + band states.  Each length is timed at tau = 1 and at tau = 0 (the same
+    library's dense path); memory is the peak device allocation over the operator path
+    (inputs, outputs, workspaces and the forward and backward calls)."""
+    from mass_adaptive_sparse_fwd_b200 import mala
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    base = synth.WORKLOADS["sinkband128k"]
+    lengths = [int(x) for x in args.sweep.split(",")] if args.sweep != "all" else SWEEP_LENGTHS
+    stream = torch.cuda.current_stream(dev)
+    rows = []
+    for L in lengths:
+        w = dataclasses.replace(base, name=f"sinkband_L{L}", L=L)
+        tr = synth.make_training(w)
+        for tau in (TAU, 0.0):
+            torch.cuda.synchronize(dev)
+            torch.cuda.empty_cache()
+            torch.cuda.reset_peak_memory_stats(dev)
+            base_bytes = torch.cuda.memory_allocated(dev)
+            Q, K, V, dO = (torch.from_numpy(tr[k]).to(dev).to(torch.bfloat16)
+                           for k in ("Q", "K", "V", "dO"))
+            B, _, H, d = Q.shape
+            Hkv = K.shape[2]
+            in_bytes = sum(t.numel() * t.element_size() for t in (Q, K, V, dO))
+            wsf = mala.alloc_workspace(mala.fwd_workspace_bytes(B, H, Hkv, L, d), dev)
+            wsb = mala.alloc_workspace(mala.bwd_workspace_bytes(B, H, Hkv, L, d), dev)
+            ws_bytes = wsf.numel() + wsb.numel()
+            torch.cuda.synchronize(dev)
+            # the conversion temporaries of the inputs are freed: start the peak here
+            torch.cuda.reset_peak_memory_stats(dev)
+            evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)]
+                   for _ in range(args.sweep_iters)]
+            for it in range(args.sweep_warmup + args.sweep_iters):
+                ev = evs[it - args.sweep_warmup] if it >= args.sweep_warmup else None
+                if ev:
+                    ev[0].record(stream)
+                O, LSE = mala.mala_fwd(Q, K, V, w.scale, tau, workspace=wsf)
+                if ev:
+                    ev[1].record(stream)
+                dQ, dK, dV = mala.mala_bwd(Q, K, V, O, LSE, dO, w.scale, tau, workspace=wsb)
+                if ev:
+                    ev[2].record(stream)
+                del O, LSE, dQ, dK, dV
+            torch.cuda.synchronize(dev)
+            for ws in (wsf, wsb):
+                err = mala.read_device_error(ws)
+                if err:
+                    raise RuntimeError(f"device error word 0x{err:x}")
+            peak = torch.cuda.max_memory_allocated(dev) - base_bytes
+            sf, sb = mala.get_stats(wsf), mala.get_stats(wsb)
+            fr = sf["retained_tiles"] / max(sf["legal_tiles"], 1)
+            br = sb["retained_tiles"] / max(sb["legal_tiles"], 1)
+            fl = fwd_bwd_flops(w, fr, br)
+            fwd = [e[0].elapsed_time(e[1]) for e in evs]
+            bwd = [e[1].elapsed_time(e[2]) for e in evs]
+            tot = [a + b for a, b in zip(fwd, bwd)]
+            rows.append({
+                "L": L, "tau": tau,
+                "fwd_ms": statistics.mean(fwd), "bwd_ms": statistics.mean(bwd),
+                "fwd_bwd_ms": statistics.mean(tot), "fwd_bwd_median_ms": statistics.median(tot),
+                "executed_tflops": (fl["fwd_exec"] + fl["bwd_exec"]) / statistics.mean(tot) / 1e9,
+                "dense_eq_tflops": (fl["fwd_dense_eq"] + fl["bwd_dense_eq"]) /
+                                   statistics.mean(tot) / 1e9,
+                "retained": {"fwd_tiles": fr, "bwd_tiles": br},
+                "peak_mem_mb": peak / 2**20,
+                "inputs_mb": in_bytes / 2**20,
+                "workspace_mb": ws_bytes / 2**20,
+                "operator_mem_mb": (peak - in_bytes) / 2**20,
+            })
+            del Q, K, V, dO, wsf, wsb
+    print(json.dumps({
+        "sweep": "operator latency and memory (fwd+bwd)",
+        "workload": "sink + band states, B=1, H=8, H_kv=1, d=128 (one rank of 8-way head "
+                    "sharding of a 64/8-head model), bf16",
+        "protocol": f"{args.sweep_warmup} warm-up + {args.sweep_iters} timed iterations per "
+                    "(L, tau), CUDA events on the launching stream, L2 not flushed; peak = "
+                    "max allocated over the operator path above the allocation before it",
+        "rows": rows}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -881,9 +970,17 @@ def main():
                     help="training workload of the step (default: the 32K headline shape)")
     ap.add_argument("--profile-case", choices=("headline", "skip", "bench32k"),
                     help="run the kernels once on a mid-size case for an ncu capture and exit")
+    ap.add_argument("--sweep", metavar="all|L1,L2,...",
+                    help="operator latency and peak memory across sequence lengths (one GPU; "
+                         "prints one JSON line and exits)")
+    ap.add_argument("--sweep-warmup", type=int, default=25)
+    ap.add_argument("--sweep-iters", type=int, default=100)
     args = ap.parse_args()
     if args.profile_case:
         profile_case(args.profile_case)
+        return
+    if args.sweep:
+        run_sweep(args)
         return
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

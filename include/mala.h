@@ -128,7 +128,11 @@ mala_status mala_fwd_varlen(const void* Q, const void* K, const void* V, void* O
  * Algorithm 2 and A.1 (fused backward execution).  O and LSE are the forward's
  * outputs; D = rowsum(O * dO) is formed inside.  dQ, dK, dV are fully written (not
  * accumulated); dK / dV sum the contributions of the H / H_kv query heads of each KV
- * head.  The workspace holds a float32 dQ accumulator [B,L,H,d] and D [B,H,L].
+ * head.  The workspace holds a float32 dQ accumulator [B,L,H,d] and D [B,H,L]; for
+ * bf16 problems with few work units (B * H_kv * (L/128 + 1) below 592, e.g. one KV head
+ * up to 64K tokens) it also holds float32 dK and dV accumulators [B,L,H_kv,d]: the query
+ * heads of a KV head are then split over several CTAs, which add their dK / dV shares.
+ * mala_bwd_workspace_bytes accounts for all of it.
  */
 mala_status mala_bwd(const void* Q, const void* K, const void* V, const void* O,
                      const float* LSE, const void* dO, void* dQ, void* dK, void* dV, int B,

@@ -7,10 +7,16 @@
 //   1. mala_bwd_prep:  D_q = rowsum(O_q * dO_q) (fp32) and zeroing of the fp32 dQ
 //                      accumulator (the softmax-backward term of Algorithm 2).
 //   2. mala_bwd_kernel (below): key-major, one persistent CTA per SM pulling units
-//                      (b, KV head g, key block j) heaviest first (small j); within a
-//                      unit the G query heads of the group and the query blocks
-//                      i = j, j+1, ... are visited in ascending order (A.1).
-//   3. mala_bwd_dq:    dQ = bf16(dQ accumulator).
+//                      (b, KV head g, key block j, head part) heaviest first (small j);
+//                      within a unit the part's query heads of the group and the query
+//                      blocks i = j, j+1, ... are visited in ascending order (A.1).
+//   3. mala_bwd_dq:    dQ = bf16(dQ accumulator) (and dK, dV likewise when split).
+//
+// Head parts: a unit normally carries all G query heads of its KV head and stores dK_j
+// and dV_j itself.  When a problem has few units (few KV heads and short sequences: the
+// j = 0 unit holds G T tiles and alone sets the kernel's length), the G heads are split
+// into P parts (P a power of two dividing G, chosen from the shape alone); each part's
+// unit adds its dK_j / dV_j share into fp32 accumulators, converted to bf16 at the end.
 //
 // Per tile (key block j, query block i of head h) the score tile S^T = K_j Q_i^T is
 // always recomputed.  The offline test of Eq. (4): the tile is retained iff some legal
@@ -70,12 +76,15 @@ struct BwdCfg {
 
 struct BwdParams {
   int B, H, Hkv, L, T, G, n_units;
+  int P, Gp;             // head parts per (b, g, j) and query heads per part (G = P Gp)
   float scale, scale_log2, log2_tau;
   const float* LSE;      // [B, H, L] natural log
   const float* Dsum;     // [B, H, L]
   float* dQacc;          // [B, L, H, D] fp32
   __nv_bfloat16* dK;     // [B, L, Hkv, D]
   __nv_bfloat16* dV;
+  float* dKacc;          // [B, L, Hkv, D] fp32 accumulators when P > 1 (scaled), else null
+  float* dVacc;
   uint8_t* tile_mask;    // [B, H, T, T] or null
   float* tile_margin;    // [B, H, T, T] debug margins (natural log) or null
   unsigned long long* stats;  // call statistics (kStatsOffset) or null
@@ -110,17 +119,18 @@ static_assert(BwdCfg<128>::SMEM + sizeof(BwdShared) <= 232448, "backward smem bu
 static_assert(BwdCfg<64>::SMEM + sizeof(BwdShared) <= 232448, "backward smem budget");
 
 struct BUnit {
-  int b, g, j, ntiles;  // tiles = G heads x (T - j) query blocks
+  int b, g, j, part, ntiles;  // tiles = Gp heads x (T - j) query blocks
 };
 
 __device__ __forceinline__ BUnit decode_bunit(const BwdParams& p, int u) {
   BUnit w;
-  const int nbg = p.B * p.Hkv;
-  w.j = u / nbg;
-  const int r = u % nbg;
-  w.b = r / p.Hkv;
-  w.g = r % p.Hkv;
-  w.ntiles = p.G * (p.T - w.j);
+  const int nbgp = p.B * p.Hkv * p.P;
+  w.j = u / nbgp;
+  const int r = u % nbgp;
+  w.part = r % p.P;
+  w.g = (r / p.P) % p.Hkv;
+  w.b = r / (p.P * p.Hkv);
+  w.ntiles = p.Gp * (p.T - w.j);
   return w;
 }
 
@@ -128,7 +138,7 @@ __device__ __forceinline__ BUnit decode_bunit(const BwdParams& p, int u) {
 __device__ __forceinline__ void tile_hi(const BwdParams& p, const BUnit& w, int n, int& h,
                                         int& i) {
   const int per = p.T - w.j;
-  h = w.g * p.G + n / per;
+  h = w.g * p.G + w.part * p.Gp + n / per;
   i = w.j + n % per;
 }
 
@@ -634,20 +644,33 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       if (got_acc) {
         const bool store = krow < p.L;
         const size_t base = ((static_cast<size_t>(w.b) * p.L + (store ? krow : 0)) * p.Hkv + w.g) * D;
+        const bool split = p.dKacc != nullptr;  // head parts: add this part's share
 #pragma unroll
         for (int which = 0; which < 2; ++which) {
           __nv_bfloat16* dst = (which == 0 ? p.dV : p.dK) + base;
+          float* accd = split ? (which == 0 ? p.dVacc : p.dKacc) + base : nullptr;
           const uint32_t src = (which == 0 ? tdV : tdK) + lane_off;
+          const float sc = (which == 1) ? p.scale : 1.f;  // dK = scale * dS^T Q
 #pragma unroll
           for (int a = 0; a < D / 32; ++a) {
             uint32_t o[32];
             tmem_ld32(src + a * 32, o);
             tmem_wait_ld();
+            if (split) {
+              if (store && valid_acc) {
+#pragma unroll
+                for (int e4 = 0; e4 < 8; ++e4) {
+                  const float* f = reinterpret_cast<const float*>(o) + e4 * 4;
+                  atomicAdd(reinterpret_cast<float4*>(accd + a * 32 + e4 * 4),
+                            make_float4(f[0] * sc, f[1] * sc, f[2] * sc, f[3] * sc));
+                }
+              }
+              continue;
+            }
 #pragma unroll
             for (int e8 = 0; e8 < 4; ++e8) {
               uint4 pk;
               const float* f = reinterpret_cast<const float*>(o) + e8 * 8;
-              const float sc = (which == 1) ? p.scale : 1.f;  // dK = scale * dS^T Q
               if (valid_acc) {
                 pk.x = pack_bf16(f[0] * sc, f[1] * sc);
                 pk.y = pack_bf16(f[2] * sc, f[3] * sc);
@@ -724,11 +747,31 @@ __global__ void __launch_bounds__(256) mala_bwd_dq(const float* __restrict__ acc
 
 }  // namespace
 
+// Head parts of a backward unit (a function of the shape alone, so that the workspace
+// query and the launch agree): the G heads are halved while the problem has fewer than
+// kPartsTarget (b, g, part) x (T + 1) work units, i.e. while the heaviest unit (key block 0,
+// Gp T tiles) would exceed about half of a 148-SM share of the legal tiles.
+constexpr long long kPartsTarget = 4 * 148;
+
+int bwd_head_parts(int B, int H, int Hkv, int L) {
+  const int G = H / Hkv;
+  const long long T = (L + kTile - 1) / kTile;
+  int P = 1;
+  while (P < G && G % (2 * P) == 0 &&
+         static_cast<long long>(B) * Hkv * (T + 1) * P < kPartsTarget)
+    P *= 2;
+  return P;
+}
+
 size_t bwd_workspace_bytes(int B, int H, int Hkv, int L, int d, int dtype) {
-  (void)Hkv; (void)dtype;
   const size_t acc = static_cast<size_t>(B) * L * H * d * sizeof(float);
   const size_t dsum = static_cast<size_t>(B) * H * L * sizeof(float);
-  return kWorkspaceHeader + ((acc + 255) / 256) * 256 + ((dsum + 255) / 256) * 256;
+  size_t bytes = kWorkspaceHeader + ((acc + 255) / 256) * 256 + ((dsum + 255) / 256) * 256;
+  if (dtype != MALA_FP32 && bwd_head_parts(B, H, Hkv, L) > 1) {
+    const size_t kv = static_cast<size_t>(B) * L * Hkv * d * sizeof(float);
+    bytes += 2 * ((kv + 255) / 256) * 256;  // dK, dV accumulators
+  }
+  return bytes;
 }
 
 mala_status fp32_bwd(const float* Q, const float* K, const float* V, const float* O,
@@ -795,8 +838,21 @@ mala_status bwd_dispatch(const void* Q, const void* K, const void* V, const void
     return MALA_ERR_CUDA;
   uint32_t* hdr = reinterpret_cast<uint32_t*>(ws);
   const size_t acc_bytes = static_cast<size_t>(B) * L * H * d * sizeof(float);
+  const size_t dsum_bytes = static_cast<size_t>(B) * H * L * sizeof(float);
   float* dQacc = reinterpret_cast<float*>(ws + kWorkspaceHeader);
   float* Dsum = reinterpret_cast<float*>(ws + kWorkspaceHeader + ((acc_bytes + 255) / 256) * 256);
+  const int P = bwd_head_parts(B, H, Hkv, L);
+  const size_t kv_bytes = static_cast<size_t>(B) * L * Hkv * d * sizeof(float);
+  float* dKacc = nullptr;
+  float* dVacc = nullptr;
+  if (P > 1) {
+    uint8_t* kv0 = ws + kWorkspaceHeader + ((acc_bytes + 255) / 256) * 256 +
+                   ((dsum_bytes + 255) / 256) * 256;
+    dKacc = reinterpret_cast<float*>(kv0);
+    dVacc = reinterpret_cast<float*>(kv0 + ((kv_bytes + 255) / 256) * 256);
+    if (cudaMemsetAsync(kv0, 0, 2 * ((kv_bytes + 255) / 256) * 256, stream) != cudaSuccess)
+      return MALA_ERR_CUDA;
+  }
   CUtensorMap tdq;
   if (!make_f32_reduce_map(&tdq, dQacc, d, H, L, B)) return MALA_ERR_CUDA;
   if (cudaMemsetAsync(hdr + kHdrSched0, 0, 3 * sizeof(uint32_t), stream) != cudaSuccess)
@@ -814,13 +870,16 @@ mala_status bwd_dispatch(const void* Q, const void* K, const void* V, const void
   if (cudaGetLastError() != cudaSuccess) return MALA_ERR_CUDA;
   BwdParams p;
   p.B = B; p.H = H; p.Hkv = Hkv; p.L = L; p.T = T; p.G = H / Hkv;
-  p.n_units = T * B * Hkv;
+  p.P = P; p.Gp = p.G / P;
+  p.n_units = T * B * Hkv * P;
   p.scale = scale;
   p.scale_log2 = scale * kLog2e;
   p.log2_tau = (tau > 0.f) ? std::log2(tau) : -INFINITY;
   p.LSE = LSE; p.Dsum = Dsum; p.dQacc = dQacc;
   p.dK = static_cast<__nv_bfloat16*>(dK);
   p.dV = static_cast<__nv_bfloat16*>(dV);
+  p.dKacc = dKacc;
+  p.dVacc = dVacc;
   p.tile_mask = tile_mask;
   p.tile_margin = tile_margin;
   p.stats = reinterpret_cast<unsigned long long*>(ws + kStatsOffset);
@@ -839,6 +898,14 @@ mala_status bwd_dispatch(const void* Q, const void* K, const void* V, const void
   const long long n4 = rows * d / 4;
   mala_bwd_dq<<<static_cast<unsigned>((n4 + 255) / 256), 256, 0, stream>>>(
       dQacc, static_cast<__nv_bfloat16*>(dQ), n4, scale);
+  if (P > 1) {
+    // the dK accumulator already holds the scale
+    const long long kv4 = static_cast<long long>(B) * L * Hkv * d / 4;
+    mala_bwd_dq<<<static_cast<unsigned>((kv4 + 255) / 256), 256, 0, stream>>>(
+        dKacc, static_cast<__nv_bfloat16*>(dK), kv4, 1.f);
+    mala_bwd_dq<<<static_cast<unsigned>((kv4 + 255) / 256), 256, 0, stream>>>(
+        dVacc, static_cast<__nv_bfloat16*>(dV), kv4, 1.f);
+  }
   return cudaGetLastError() == cudaSuccess ? MALA_OK : MALA_ERR_CUDA;
 }
 

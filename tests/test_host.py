@@ -120,6 +120,29 @@ def test_workspace_sizes_and_split_rule(lib):
     assert lib.decode_workspace_bytes(1, 4, 2, 256, 128, 0, 5) == 0  # 5 splits > 2 tiles
 
 
+def _round256(n):
+    return (n + 255) // 256 * 256
+
+
+def test_bwd_workspace_head_parts(lib):
+    """The backward splits a unit's query heads into parts when a problem has few units
+    (few KV heads, short sequences); the parts add dK / dV into two fp32 accumulators that
+    the workspace then holds.  Many units (the 32K 32/8-head shape, the 128K 8/1-head
+    shape): no split, no accumulators."""
+    def base(B, H, Hkv, L, d):
+        return 256 + _round256(B * L * H * d * 4) + _round256(B * H * L * 4)
+
+    def kv(B, Hkv, L, d):
+        return 2 * _round256(B * L * Hkv * d * 4)
+
+    for shape in [(1, 32, 8, 32768, 128), (1, 8, 1, 131072, 128), (2, 6, 2, 300, 64),
+                  (1, 2, 2, 384, 128)]:  # enough units, or G odd / G = 1: one part
+        assert lib.bwd_workspace_bytes(*shape) == base(*shape)
+    for B, H, Hkv, L, d in [(1, 8, 1, 32768, 128), (1, 8, 1, 1024, 128), (1, 16, 4, 8192, 128),
+                            (2, 8, 2, 1024, 128), (1, 4, 1, 2048, 64)]:
+        assert lib.bwd_workspace_bytes(B, H, Hkv, L, d) == base(B, H, Hkv, L, d) + kv(B, Hkv, L, d)
+
+
 @pytest.mark.parametrize("shape,expect", [
     ((4, 32, 8, 131072), 9),    # 288 units: two full waves of 228 tiles per CTA
     ((4, 32, 8, 32768), 4),     # one wave of 128 CTAs
