@@ -5,7 +5,8 @@
 //
 // One persistent CTA per SM pulls work units from an atomic counter.  A unit is one
 // 128-row query block i of two query heads that share a KV head (two "slots"), so both
-// slots stream the same K_j / V_j tiles; units are numbered heaviest first (largest i).
+// slots stream the same K_j / V_j tiles; units are numbered heaviest first (largest i)
+// within a KV head.
 // Within a unit the key blocks are visited from the block of the unit's last query
 // position down to 0 (diagonal first).  For chunked prefill (§2.3: the forward serves
 // inference prefill) the L query rows are the last L of Lk key positions: row q sits at
@@ -44,6 +45,10 @@
 // The forward is tensor-core bound and deciding first would put the V latency on the
 // critical path of every retained tile; the skipped work is the exponentials and the
 // PV MMA.  (Decode, which is bandwidth bound, gates its V loads on the decision.)
+//
+// Units are numbered KV head slowest and heaviest first within a head, so that the CTAs
+// running together share one head's K and V in L2 (on skipped tiles the forward waits on
+// K/V loads through the two-stage ring, and L2 hits shorten them).
 
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -120,11 +125,14 @@ __device__ __forceinline__ Unit decode_unit(const FwdParams& p, int u) {
     w.L = e.L;
     w.off = e.off;
   } else {
-    const int nbg = p.B * p.Hkv * p.npairs;
-    w.i = p.T - 1 - u / nbg;
-    r = u % nbg;
-    w.b = r / (p.Hkv * p.npairs);
-    w.g = (r / p.npairs) % p.Hkv;
+    // KV head slowest: the CTAs that run together share one head's K and V in L2;
+    // heaviest first (largest i) within a head
+    const int nbp = p.B * p.npairs;
+    const int upg = nbp * p.T;
+    w.g = u / upg;
+    r = u % upg;
+    w.i = p.T - 1 - r / nbp;
+    w.b = (r % nbp) / p.npairs;
     hp = r % p.npairs;
     w.qrow0 = 0;
     w.krow0 = 0;
