@@ -7,7 +7,9 @@
 //   1. mala_bwd_prep:  D_q = rowsum(O_q * dO_q) (fp32) and zeroing of the fp32 dQ
 //                      accumulator (the softmax-backward term of Algorithm 2).
 //   2. mala_bwd_kernel (below): key-major, one persistent CTA per SM pulling units
-//                      (b, KV head g, key block j, head part) heaviest first (small j);
+//                      (b, KV head g, key block j, head part), KV head slowest and
+//                      heaviest first (small j) within a head, so that the CTAs running
+//                      together share one group's Q, dO and dQ accumulator in L2;
 //                      within a unit the part's query heads of the group and the query
 //                      blocks i = j, j+1, ... are visited in ascending order (A.1).
 //   3. mala_bwd_dq:    dQ = bf16(dQ accumulator) (and dK, dV likewise when split).
@@ -124,12 +126,14 @@ struct BUnit {
 
 __device__ __forceinline__ BUnit decode_bunit(const BwdParams& p, int u) {
   BUnit w;
-  const int nbgp = p.B * p.Hkv * p.P;
-  w.j = u / nbgp;
-  const int r = u % nbgp;
+  // KV head slowest, heaviest first (small j) within a head
+  const int nbp = p.B * p.P;
+  const int upg = nbp * p.T;
+  w.g = u / upg;
+  const int r = u % upg;
+  w.j = r / nbp;
+  w.b = (r % nbp) / p.P;
   w.part = r % p.P;
-  w.g = (r / p.P) % p.Hkv;
-  w.b = r / (p.P * p.Hkv);
   w.ntiles = p.Gp * (p.T - w.j);
   return w;
 }
