@@ -99,6 +99,9 @@ def check_bwd(orc, mala, w, inp, tau, kv_units=None, q_units=None, flags=0, max_
     dict(B=1, H=4, Hkv=2, L=256, d=128, structure="peaked"),
     dict(B=2, H=6, Hkv=2, L=300, d=64, structure="normal"),
     dict(B=1, H=2, Hkv=2, L=384, d=128, structure="peaked"),
+    # few units: the query heads of a KV head are split over 4 CTAs, which add their dK /
+    # dV shares in fp32 (ragged length, d = 64)
+    dict(B=2, H=8, Hkv=2, L=333, d=64, structure="peaked"),
 ])
 def test_bwd_small(orc, mala, shape, tau):
     w, inp = synth.small_training(**shape)
