@@ -876,7 +876,9 @@ def run_sweep(args):
     H_kv=1, d=128; the sharded ranks run independent problems of this shape), on the
     sink + band states.  Each length is timed at tau = 1 and at tau = 0 (the same
     library's dense path); memory is the peak device allocation over the operator path
-    (inputs, outputs, workspaces and the forward and backward calls)."""
+    (inputs, outputs, workspaces and the forward and backward calls).  Decode is timed on
+    the same rank shape at batch 1: the last position's query heads against the L-token
+    K/V cache, with its own peak allocation (cache, query, outputs, workspace)."""
     from mass_adaptive_sparse_fwd_b200 import mala
 
     dev = torch.device("cuda", 0)
@@ -923,6 +925,32 @@ def run_sweep(args):
                 if err:
                     raise RuntimeError(f"device error word 0x{err:x}")
             peak = torch.cuda.max_memory_allocated(dev) - base_bytes
+            # decode: one query per head (the last position) against the whole K/V cache;
+            # its peak = the cache (already resident) plus what the decode path allocates
+            torch.cuda.synchronize(dev)
+            torch.cuda.reset_peak_memory_stats(dev)
+            dec_start = torch.cuda.memory_allocated(dev)
+            q = Q[:, L - 1].contiguous()
+            S = mala.decode_num_splits(B, H, Hkv, L)
+            wsd = mala.alloc_workspace(mala.decode_workspace_bytes(B, H, Hkv, L, d, 0, S), dev)
+            dev_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)]
+                      for _ in range(args.sweep_iters)]
+            for it in range(args.sweep_warmup + args.sweep_iters):
+                ev = dev_ev[it - args.sweep_warmup] if it >= args.sweep_warmup else None
+                if ev:
+                    ev[0].record(stream)
+                Od, Ld = mala.mala_decode(q, K, V, w.scale, tau, num_splits=S, workspace=wsd)
+                if ev:
+                    ev[1].record(stream)
+                del Od, Ld
+            torch.cuda.synchronize(dev)
+            if mala.read_device_error(wsd):
+                raise RuntimeError("decode device error")
+            sd = mala.get_stats(wsd)
+            dec_us = [1e3 * e[0].elapsed_time(e[1]) for e in dev_ev]
+            dec_peak = (torch.cuda.max_memory_allocated(dev) - dec_start +
+                        (K.numel() + V.numel()) * 2)
+            del wsd, q
             sf, sb = mala.get_stats(wsf), mala.get_stats(wsb)
             fr = sf["retained_tiles"] / max(sf["legal_tiles"], 1)
             br = sb["retained_tiles"] / max(sb["legal_tiles"], 1)
@@ -942,6 +970,10 @@ def run_sweep(args):
                 "inputs_mb": in_bytes / 2**20,
                 "workspace_mb": ws_bytes / 2**20,
                 "operator_mem_mb": (peak - in_bytes) / 2**20,
+                "decode": {"us": statistics.mean(dec_us), "median_us": statistics.median(dec_us),
+                           "splits": S,
+                           "v_tiles_retained": sd["v_tiles_loaded"] / max(sd["legal_tiles"] / H * Hkv, 1),
+                           "peak_mem_mb": dec_peak / 2**20},
             })
             del Q, K, V, dO, wsf, wsb
     print(json.dumps({
