@@ -97,6 +97,7 @@ struct DecShared {
   // per-warp tile maxima and row sums, [warp][head], double-buffered by tile parity
   float rmax[2][8][8];
   float rsum[2][8][8];
+  float mz[8], mw[8];                 // merge: per head max_s z_s and sum_s e^(z_s - max)
   uint32_t last_flag;
   uint32_t abort_flag;
 };
@@ -547,21 +548,52 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS, 1)
       named_bar_sync(1, NT);
       if (sh.last_flag) {
         __threadfence();
+        // The other CTAs' partials are read from L2 (ld.global.cg).  First one warp per
+        // head: z = log sum_s e^(z_s), from lane-strided loads and shuffles.
+        for (int hh = warp; hh < G; hh += CW) {
+          const size_t row = static_cast<size_t>(b) * p.H + g * G + hh;
+          const float* pz = p.part_z + row * p.S;
+          float zmax = NEG_INF;
+          for (int ss = lane; ss < p.S; ss += 32) zmax = fmaxf(zmax, __ldcg(pz + ss));
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1)
+            zmax = fmaxf(zmax, __shfl_xor_sync(0xffffffffu, zmax, o));
+          float wsum = 0.f;
+          for (int ss = lane; ss < p.S; ss += 32) wsum += __expf(__ldcg(pz + ss) - zmax);
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, o);
+          if (lane == 0) {
+            sh.mz[hh] = zmax;
+            sh.mw[hh] = wsum;
+            p.LSE[row] = zmax + __logf(wsum);
+          }
+        }
+        named_bar_sync(1, NT);
+        // then o = sum_s e^(z_s - z) o_s, one output element per thread and pass; the
+        // split loop's loads are independent, so several are in flight at once
         for (int i = tid; i < G * D; i += NT) {
           const int hh = i / D, dd = i % D;
           const size_t row = static_cast<size_t>(b) * p.H + g * G + hh;
-          const volatile float* pz = p.part_z + row * p.S;
-          const volatile float* po = p.part_o + row * p.S * D;
-          float zmax = NEG_INF;
-          for (int ss = 0; ss < p.S; ++ss) zmax = fmaxf(zmax, pz[ss]);
-          float wsum = 0.f, o = 0.f;
-          for (int ss = 0; ss < p.S; ++ss) {
-            const float wgt = __expf(pz[ss] - zmax);
-            wsum += wgt;
-            o += wgt * po[ss * D + dd];
+          const float* pz = p.part_z + row * p.S;
+          const float* po = p.part_o + row * p.S * D + dd;
+          const float zmax = sh.mz[hh];
+          float o0 = 0.f, o1 = 0.f;
+          int ss = 0;
+          for (; ss + 8 <= p.S; ss += 8) {
+            float zv[8], ov[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              zv[e] = __ldcg(pz + ss + e);
+              ov[e] = __ldcg(po + static_cast<size_t>(ss + e) * D);
+            }
+#pragma unroll
+            for (int e = 0; e < 8; e += 2) {
+              o0 += __expf(zv[e] - zmax) * ov[e];
+              o1 += __expf(zv[e + 1] - zmax) * ov[e + 1];
+            }
           }
-          p.O[row * D + dd] = __float2bfloat16(o / wsum);
-          if (dd == 0) p.LSE[row] = zmax + __logf(wsum);
+          for (; ss < p.S; ++ss) o0 += __expf(__ldcg(pz + ss) - zmax) * __ldcg(po + static_cast<size_t>(ss) * D);
+          p.O[row * D + dd] = __float2bfloat16((o0 + o1) / sh.mw[hh]);
         }
       }
     }
