@@ -213,8 +213,9 @@ size_t mala_decode_workspace_bytes(int B, int H, int H_kv, int Nk, int d, int dt
 /* The split count used when mala_decode is given num_splits = 0 (deterministic, host
  * only, no device query).  Among the counts that give at most two waves of units
  * (b, KV head, split) over 148 persistent CTAs, it takes the S that minimises
- * waves x (ceil(T / S) + 10): a CTA's time is its key tiles plus a fixed cost of about
- * ten tiles per unit.  Ties go to fewer splits.  Returns 0 for invalid shapes. */
+ * waves x (ceil(T / S) + 10) + S / 9: a CTA's time is its key tiles plus a fixed cost of
+ * about ten tiles per unit, and merging the S partials of a (b, KV head) costs about
+ * S / 9 tiles.  Ties go to fewer splits.  Returns 0 for invalid shapes. */
 int mala_decode_num_splits(int B, int H, int H_kv, int Nk);
 
 /* Reads the device error word of a workspace (synchronises `stream`).  *out receives
@@ -271,9 +272,10 @@ mala_status mala_set_debug(const mala_debug* dbg);
 
 const char* mala_status_string(mala_status s);
 
-/* Library version: 202 = 0.2.2 (0.2.0 added mala_fwd_prefill, mala_fwd_varlen and
+/* Library version: 203 = 0.2.3 (0.2.0 added mala_fwd_prefill, mala_fwd_varlen and
  * mala_get_stats; 0.2.1 changes the automatic decode split count, mala_decode_num_splits;
- * 0.2.2 adds mala_set_debug). */
+ * 0.2.2 adds mala_set_debug; 0.2.3 changes the automatic decode split count again, for
+ * small batches: it now accounts for the cost of merging the splits). */
 int mala_version(void);
 
 #ifdef __cplusplus

@@ -159,7 +159,7 @@ using namespace mala;
 
 extern "C" {
 
-int mala_version(void) { return 202; }
+int mala_version(void) { return 203; }
 
 const char* mala_status_string(mala_status s) {
   switch (s) {

@@ -610,10 +610,11 @@ int decode_auto_splits(int B, int Hkv, int Nk) {
   // the pipeline fill and drain, the partial write and the ticket), the fixed cost being
   // worth about 10 tiles at the HBM rate.  One SM alone streams K and V at about 1/148 of
   // the HBM rate, so a single wave of fewer CTAs is not bandwidth-starved beyond its tile
-  // count.  The rule takes the split count S <= T of at most two waves that minimises
-  // ceil(B Hkv S / 148) (ceil(T / S) + 10); ties go to fewer splits (fewer partials to
-  // merge).
-  constexpr int kSMs = 148, kUnitCostTiles = 10;
+  // count.  The last CTA of each (b, g) then merges its S partials, which adds about S / 9
+  // tiles (measured: with one KV head at batch 1 the best S grows as about 3 sqrt(T)).
+  // The rule takes the split count S <= T of at most two waves that minimises
+  // ceil(B Hkv S / 148) (ceil(T / S) + 10) + S / 9; ties go to fewer splits.
+  constexpr int kSMs = 148, kUnitCostTiles = 10, kSplitsPerMergeTile = 9;
   const int T = (Nk + kTile - 1) / kTile;
   const int bg = B * Hkv;
   int smax = (2 * kSMs) / bg;
@@ -623,7 +624,9 @@ int decode_auto_splits(int B, int Hkv, int Nk) {
   long long best_cost = -1;
   for (int s = 1; s <= smax; ++s) {
     const long long waves = (static_cast<long long>(bg) * s + kSMs - 1) / kSMs;
-    const long long cost = waves * ((T + s - 1) / s + kUnitCostTiles);
+    // in units of 1/9 tile
+    const long long cost =
+        kSplitsPerMergeTile * waves * ((T + s - 1) / s + kUnitCostTiles) + s;
     if (best_cost < 0 || cost < best_cost) {
       best_cost = cost;
       best_s = s;
