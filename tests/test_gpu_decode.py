@@ -74,6 +74,19 @@ def test_decode_small(orc, mala, shape, S, tau):
         assert (mask == 0).any()
 
 
+@pytest.mark.parametrize("tau", [0.0, 1.0])
+@pytest.mark.parametrize("S", [37, 0])
+def test_decode_batch1_many_splits(orc, mala, S, tau):
+    """One KV head at batch 1 (a rank of 8-way head sharding): many splits, so the merge
+    runs its eight-deep unrolled loop several times plus a remainder (37 splits), and the
+    automatic count of the split rule's merge term (22 at 8K)."""
+    w, inp = _planted(1, 8, 1, 8192, 128, seed=23)
+    if S == 0:
+        S = mala.decode_num_splits(1, 8, 1, 8192)
+        assert S == 22
+    check_decode(orc, mala, inp, w.scale, tau, S, name="decode_b1")
+
+
 def test_decode_always_test_flag(orc, mala):
     w, inp = _planted(2, 8, 2, 1024, 128, seed=22)
     check_decode(orc, mala, inp, w.scale, 0.0, 2, flags=1)
