@@ -102,6 +102,8 @@ def check_bwd(orc, mala, w, inp, tau, kv_units=None, q_units=None, flags=0, max_
     # few units: the query heads of a KV head are split over 4 CTAs, which add their dK /
     # dV shares in fp32 (ragged length, d = 64)
     dict(B=2, H=8, Hkv=2, L=333, d=64, structure="peaked"),
+    # one KV head of 8 query heads at 1K: every query head gets its own CTA (P = 8)
+    dict(B=1, H=8, Hkv=1, L=1024, d=128, structure="peaked"),
 ])
 def test_bwd_small(orc, mala, shape, tau):
     w, inp = synth.small_training(**shape)
